@@ -1,0 +1,430 @@
+#!/usr/bin/env python
+"""Benchmark of the per-rank mixed-precision Adam shard step on B200.
+
+    python bench.py [--gpus N --steps K --warmup W] [--workload pythia_1p4b]
+    python bench.py --impl reference ...      # the CPU oracle as the reference arm
+
+One step = one neox_shard_step call over the whole owned shard: pass 1 (ingest,
+overflow flag, global norm, loss scaler, clip coefficient) and pass 2 (AdamW on
+FP32 master/m/v + cast to the 16-bit working copy).  Inputs are resident in HBM
+(22.6 GB for the default 1.41e9-parameter shard, far above the 126 MB L2, so no
+flush is needed between steps).  Under torchrun every rank steps its own shard of
+the same size (weak scaling); the per-rank step has no data-path collective.
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Adam shard-step Gparams/s and achieved HBM GB/s (% of B200 peak), 1 GPU"
+UNIT = "Gparams/s"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SRC = os.path.join(ROOT, "mixed_precision_zero_b200", "csrc", "neox_shard.cu")
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["b200", "reference"], default="b200")
+    p.add_argument("--workload", default="pythia_1p4b")
+    p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    a = p.parse_args(argv)
+    if a.warmup < 3:
+        p.error("--warmup must be >= 3")
+    return a
+
+
+# ------------------------------------------------------------------ workload bytes
+
+def alg_bytes_per_param(K: int, acc: bool):
+    """Algorithmic HBM bytes per parameter of an applied step: (pass 1, pass 2)."""
+    p1 = 2 * K + (4 if acc else 0)
+    p2 = (4 if acc else 2 * K) + 12 + 12 + 2
+    return p1, p2
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    with open(KERNEL_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch of the update kernel from the committed ncu summary,
+    if it was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"adam_kernel_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_src = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    m_tr = re.search(r"dram_bytes_per_launch_full_size:\s*([0-9.eE+]+)", text)
+    if not (m_src and m_tr) or m_src.group(1) != kernel_source_hash():
+        return None
+    return float(m_tr.group(1))
+
+
+# ------------------------------------------------------------------ clocks (NVML)
+
+class ClockSampler:
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting",
+               0x1: "gpu_idle", 0x10: "sync_boost"}
+
+    def __init__(self, device_index: int, interval=0.05):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.interval = interval
+        self._stop = threading.Event()
+        self._thr = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.h = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(h)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                    self.h = h
+            if self.h is not None:
+                self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.nv = pynvml
+        except Exception as e:  # clocks are reported as unavailable, the run goes on
+            log(f"clock sampling unavailable: {e}")
+            self.h = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.interval)
+
+    def __enter__(self):
+        if self.h is not None:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thr:
+            self._thr.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ oracle on the host cores
+
+def cpu_sample_range(wl, size):
+    """A contiguous sample of the workload that crosses segment boundaries when
+    it has any: centred on the first non-trivial segment boundary."""
+    if wl.segments and len(wl.segments) > 1:
+        b = wl.segments[1][0]
+        lo = max(0, min(b - size // 2, wl.numel - size))
+    else:
+        lo = 0
+    return lo, min(size, wl.numel - lo)
+
+
+def sample_segments(wl, lo, n):
+    if not wl.segments:
+        return None, [("normal", 0, n)]
+    segs, inits = [], []
+    for off, cnt, wd, init in wl.segments:
+        a, b = max(off, lo), min(off + cnt, lo + n)
+        if a < b:
+            segs.append((a - lo, b - a, wd))
+            inits.append((init, a - lo, b - a))
+    return segs, inits
+
+
+def run_oracle_sample(wl, n_sample, steps, seconds, rank_seed=0):
+    """Time the single-threaded oracle on `steps` calls over a contiguous sample
+    of the workload (inputs drawn by the numpy twin of the generator, untimed)."""
+    import numpy as np
+
+    import oracle
+    import synth
+    lo, n = cpu_sample_range(wl, n_sample)
+    segs, inits = sample_segments(wl, lo, n)
+    master = synth.master_normal(n, wl.master_sigma, wl.seed + rank_seed, 0, start=lo)
+    for init, a, c in inits:
+        if init == "zero":
+            master[a:a + c] = 0
+        elif init == "one":
+            master[a:a + c] = 1
+    hp = oracle.OracleHparams(wl.beta1, wl.beta2, wl.eps, wl.clip, wl.predivide, wl.init_scale, 2.0, 1.0,
+                              wl.scale_window)
+    sh = oracle.OracleShard(master, hp, wbf16=wl.bf16, gbf16=wl.bf16, segments=segs, default_wd=wl.weight_decay)
+    grads = []
+    for k in range(wl.K):
+        if wl.grad_dist == "t3":
+            grads.append(synth.grad_t3_16(n, sh.scale, wl.seed + rank_seed, k, 1, wl.bf16, start=lo))
+        else:
+            grads.append(synth.grad_normal16(n, wl.grad_sigma, sh.scale, wl.seed + rank_seed, k, 1, wl.bf16, start=lo))
+    times = []
+    t_all = time.perf_counter()
+    for s in range(steps):
+        t0 = time.perf_counter()
+        sh.step(grads, wl.lr)
+        times.append(time.perf_counter() - t0)
+        if seconds and time.perf_counter() - t_all > seconds and s >= 0:
+            break
+    return {"n": n, "lo": lo, "times": times}
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args):
+    from synth import workloads as W
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    wl = W.ALL[args.workload]()
+    total = args.steps + args.warmup
+    per_step_budget = max(0.2, 150.0 / total)           # whole run within a few minutes
+    n_sample = int(min(1 << 24, max(1 << 16, per_step_budget / 60e-9)))
+    out = run_oracle_sample(wl, n_sample, total, 0.0)
+    times = out["times"][args.warmup:]
+    sec = sum(times)
+    value = out["n"] * len(times) / sec / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": len(times), "warmup": args.warmup, "ms_per_step": 1e3 * sec / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": wl.name, "numel": wl.numel, "grad_buffers": wl.K,
+                   "sample": f"{out['n']} contiguous elements from index {out['lo']} per step"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"{out['n']} contiguous elements of {wl.name}, {len(times)} timed steps"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ B200 arm
+
+def build_gpu_workload(wl, rank):
+    import torch
+
+    import synth
+    from mixed_precision_zero_b200 import Hparams, NeoxShard
+    n = wl.numel
+    dt = torch.bfloat16 if wl.bf16 else torch.float16
+    seed = wl.seed + 1000 * rank
+    master = torch.empty(n, dtype=torch.float32, device="cuda")
+    synth.gpu_master_normal(master, wl.master_sigma, seed)
+    for off, cnt, _, init in (wl.segments or []):
+        if init == "zero":
+            master[off:off + cnt].zero_()
+        elif init == "one":
+            master[off:off + cnt].fill_(1.0)
+    m = torch.zeros_like(master)
+    v = torch.zeros_like(master)
+    params = master.to(dt)
+    grads = []
+    for k in range(wl.K):
+        g = torch.empty(n, dtype=dt, device="cuda")
+        if wl.grad_dist == "t3":
+            synth.gpu_grad_t3_16(g, wl.init_scale, seed, k, 1, wl.bf16)
+        else:
+            synth.gpu_grad_normal16(g, wl.grad_sigma, wl.init_scale, seed, k, 1, wl.bf16)
+        grads.append(g)
+    hp = Hparams(wl.beta1, wl.beta2, wl.eps, wl.clip, wl.predivide, wl.init_scale, 2.0, 1.0, wl.scale_window)
+    shard = NeoxShard(master, m, v, hp, wdtype=dt, gdtype=dt, segments=wl.seg_table(),
+                      weight_decay=wl.weight_decay, max_grads=wl.K)
+    torch.cuda.synchronize()
+    return shard, grads, params, (master, m, v)
+
+
+def run_b200(args):
+    import torch
+    import torch.distributed as dist
+
+    from synth import workloads as W
+    ws, rank, local = dist_env()
+    if ws != args.gpus:
+        log(f"note: --gpus {args.gpus} but WORLD_SIZE {ws}; using WORLD_SIZE")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    wl = W.ALL[args.workload]()
+    shard, grads, params, state = build_gpu_workload(wl, rank)
+    acc = wl.K >= 5
+    p1b, p2b = alg_bytes_per_param(wl.K, acc)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        res = shard.step(grads, params, wl.lr)
+    t_before = shard.get_state()[2]
+    shard.reset_profile()
+    shard.set_profiling(True)
+    launches0 = shard.profile().launches
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            res = shard.step(grads, params, wl.lr)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    ms_local = ev0.elapsed_time(ev1)
+    prof = shard.profile()
+    launches = prof.launches - launches0
+    applied = shard.get_state()[2] - t_before
+    assert applied == args.steps, f"{args.steps - applied} timed steps were skipped (overflow)"
+    shard.set_profiling(False)
+
+    ms = max_over_ranks(ms_local, dev)
+    total_params = sum_over_ranks(float(wl.numel), dev)
+    ms_step = ms / args.steps
+    value = total_params * args.steps / (ms * 1e-3) / 1e9
+    p1_ms = prof.grad_pass_ms / prof.steps
+    p2_ms = prof.update_pass_ms / prof.steps
+    peak, peak_kind = hbm_peak()
+    achieved = p2b * wl.numel / (p2_ms * 1e-3) / 1e9
+    step_gbs = (p1b + p2b) * wl.numel / (ms_local / args.steps * 1e-3) / 1e9
+    traffic = recorded_traffic(args.workload)
+
+    # end to end through the public API: grads from pinned host memory each step
+    host_grads = [g.cpu().pin_memory() for g in grads]
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if ws > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        for g, hg in zip(grads, host_grads):
+            g.copy_(hg, non_blocking=True)
+        res = shard.step(grads, params, wl.lr)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    e2e_value = total_params * args.e2e_steps / (e2e_ms * 1e-3) / 1e9
+    h2d = sum(g.numel() * g.element_size() for g in grads)
+    d2h = 64  # the step's device scalar block, read into pinned memory by every call
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        out = run_oracle_sample(wl, 1 << 25, 50, args.cpu_seconds)
+        sec = sum(out["times"])
+        cpu = {"value": out["n"] * len(out["times"]) / sec / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"{len(out['times'])} steps over {out['n']} contiguous elements of {wl.name} "
+                         f"(from index {out['lo']}), single-threaded oracle"}
+
+    clk = clocks.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": wl.name, "numel_per_rank": wl.numel, "segments": len(wl.segments or [1]),
+                   "grad_buffers": wl.K, "weights": "bf16" if wl.bf16 else "fp16",
+                   "state": "fp32 master/m/v", "l2": "inputs 22.6 GB per rank >> 126 MB L2; no flush",
+                   "parallelism": f"{ws} independent shard(s), one per GPU"},
+        "hbm": {"step_gbs": step_gbs, "step_frac": step_gbs / peak, "bytes_per_param": p1b + p2b,
+                "peak_gbs": peak, "peak_kind": peak_kind},
+        "roofline": {"bound": "hbm", "kernel": "adam_kernel (pass 2)", "achieved": achieved, "peak": peak,
+                     "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
+                     "traffic": traffic, "alg_bytes_per_launch": p2b * wl.numel,
+                     "avg_launch_ms": p2_ms, "grad_pass_avg_ms": p1_ms},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": args.e2e_steps},
+        "gpu_launches": launches,
+        "clocks": clk,
+        "impl": "b200",
+    }
+    if cpu:
+        line["cpu_baseline"] = cpu
+    shard.close()
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_b200(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

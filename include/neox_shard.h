@@ -1,0 +1,191 @@
+/*
+ * neox_shard.h -- C ABI of libneoxshard.so: the per-rank mixed-precision
+ * optimizer step over an owned flat shard, as hand-written CUDA for sm_100a.
+ *
+ * What the step computes (pages, by title and section):
+ *  - "GPT-NeoX: how it opened the door to democratised 100B-scale training"
+ *    (ainews.cool), section "技术深度解析" (technical deep-dive): with ZeRO
+ *    stage 1 the optimizer state is partitioned across the data-parallel
+ *    ranks and each device updates only the shard it owns.  One handle of
+ *    this library is one such shard on one GPU.
+ *  - "OPT: Open Pre-trained Transformer Language Models" (ai-papers.xuzou.cn
+ *    summary), section "计算设置" (compute setup): Adam state in FP32, sharded;
+ *    weights in FP16; dynamic loss scaling against underflow.
+ *  - same page, section "瓶颈" (bottlenecks): about 16 bytes of model state
+ *    per parameter (FP16 weight + FP16 grad + FP32 master, m, v).
+ *  - same page, section "方法适配" (method adaptation): a gradient pre-divide
+ *    factor, global-norm gradient clipping at 1.0 or 0.3, and resetting the
+ *    dynamic loss scaler / restarting from a checkpoint where it is healthy.
+ *  - The pages never write Adam out; the update is the textbook AdamW
+ *    (Loshchilov & Hutter, decoupled weight decay) with bias correction.
+ *
+ * One call of neox_shard_step, for K gradient buffers g_0..g_{K-1} (16-bit,
+ * numel elements each) carrying the current loss scale S:
+ *   1. g_i = fl32( (sum_k fl32(g_k,i * fl32(1/predivide))) * fl32(1/(post*S)) ),
+ *      post = K/predivide, the sum taken in buffer order in FP32;
+ *   2. overflow = any g_i not finite (or the norm not finite);
+ *   3. norm = sqrt(sum_i g_i^2)  (pre-clip, unscaled);
+ *   4. loss scaler: overflow -> S = max(S/factor, min_scale), counter = 0, skip;
+ *      applied -> counter+1, at scale_window S = S*factor (if finite), counter = 0;
+ *   5. unless skipped: t = t+1; c = clip/(norm+1e-6) if that is < 1 (else 1);
+ *      for every element: gh = g*c; m = b1*m + (1-b1)*gh; v = b2*v + (1-b2)*gh*gh;
+ *      p = p*(1 - lr*wd_seg) - (lr/bc1) * m / (sqrt(v)/sqrt(bc2) + eps),
+ *      bc1 = 1-b1^t, bc2 = 1-b2^t; w = RNE16(p).
+ *
+ * Threading: a handle is used by one host thread at a time.  Different
+ * handles are independent.  All functions are host functions.
+ */
+#ifndef NEOX_SHARD_H
+#define NEOX_SHARD_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NEOX_OK = 0,
+    NEOX_ERR_INVALID_ARGUMENT = 1, /* nothing launched, no state changed      */
+    NEOX_ERR_CUDA = 2,             /* a CUDA call failed; see neox_last_error */
+    NEOX_ERR_OUT_OF_MEMORY = 3,    /* device or pinned allocation failed      */
+    NEOX_ERR_UNSUPPORTED = 4       /* e.g. the device is not sm_100           */
+} neox_status;
+
+typedef enum { NEOX_FP16 = 0, NEOX_BF16 = 1 } neox_dtype;
+
+/* A run of elements [offset, offset+numel) with its own weight decay (biases
+ * and LayerNorm parameters typically use 0).  A table must be sorted by
+ * offset and tile [0, numel) exactly, each segment non-empty. */
+typedef struct {
+    uint64_t offset;
+    uint64_t numel;
+    float weight_decay;
+} neox_segment;
+
+typedef struct {
+    float beta1, beta2;   /* in [0, 1)                                      */
+    float eps;            /* >= 0                                           */
+    float clip_norm;      /* global-norm clip; <= 0 disables clipping       */
+    float predivide;      /* > 0; each buffer is scaled by 1/predivide
+                             before the sum, the sum by predivide/K after    */
+    float init_scale;     /* > 0: the loss scale at create                  */
+    float scale_factor;   /* >= 1: backoff divisor and growth multiplier    */
+    float min_scale;      /* >= 0: floor of the scale after a backoff       */
+    int32_t scale_window; /* >= 1: applied steps between growths            */
+} neox_hparams;
+
+/* The shard.  numel may be 0 (a rank that owns nothing still takes part in
+ * the scaler).  master / exp_avg / exp_avg_sq are caller-owned device FP32
+ * arrays of numel elements (NULL allowed only when numel == 0); they must be
+ * 4-byte aligned and must outlive the handle.  The caller initialises them
+ * (typically m = v = 0) and the 16-bit working weights to RNE16(master). */
+typedef struct {
+    uint64_t numel;
+    neox_dtype wdtype;            /* working-weight type (params of the step) */
+    neox_dtype gdtype;            /* gradient type                            */
+    const neox_segment* segs;     /* host array; NULL = one segment [0,numel)  */
+    int32_t nsegs;
+    float default_weight_decay;   /* weight decay when segs == NULL           */
+    float* master;
+    float* exp_avg;
+    float* exp_avg_sq;
+    int32_t max_grads;            /* largest K the caller will pass (0 = 1);
+                                     K >= 5 makes create reserve numel*4 bytes
+                                     of FP32 scratch so pass 2 reads one FP32
+                                     sum instead of re-reading K buffers       */
+} neox_shard_desc;
+
+typedef struct {
+    int32_t overflow;          /* 1: non-finite gradient; the step was skipped */
+    float grad_norm;           /* pre-clip L2 norm of the unscaled gradient;
+                                  +inf when overflow                          */
+    float clip_coef;           /* coefficient applied to the gradient (1 = no
+                                  clipping); 0 when overflow                  */
+    float loss_scale;          /* S that this step's gradients carried        */
+    float loss_scale_next;     /* S to multiply the next loss by              */
+    int32_t good_steps;        /* scaler counter after this step              */
+    int64_t applied_steps;     /* t after this step                           */
+} neox_step_result;
+
+typedef struct neox_shard neox_shard;
+
+/* Create a handle for one shard on CUDA device `device`.
+ * Validates desc and hp (NEOX_ERR_INVALID_ARGUMENT on any violation, nothing
+ * allocated), checks the device is compute capability 10.x (else
+ * NEOX_ERR_UNSUPPORTED), copies the segment table to the device and allocates
+ * the handle's scratch: a few KB of per-block partial sums, a 64-byte device
+ * scalar block, a pinned 64-byte result slot, and (max_grads >= 5) an FP32
+ * accumulation buffer of numel elements.  The loss scale starts at
+ * hp->init_scale with zero counters.  *out is set only on NEOX_OK. */
+neox_status neox_shard_create(const neox_shard_desc* desc, const neox_hparams* hp,
+                              int device, neox_shard** out);
+
+/* One optimizer step (steps 1-5 above) on cuda_stream (a cudaStream_t; NULL =
+ * the legacy default stream).
+ *   grads:     host array of num_grads DEVICE pointers, each to numel 16-bit
+ *              gradients of desc->gdtype, 2-byte aligned, read only;
+ *   num_grads: K in [1, 64];
+ *   params:    DEVICE pointer to numel 16-bit working weights of
+ *              desc->wdtype, 2-byte aligned, written only when the step is
+ *              applied; must not overlap any other array;
+ *   lr:        learning rate of this step, finite and >= 0;
+ *   out:       host result, filled on NEOX_OK.
+ * Arrays may start at any element offset: when every array has the same
+ * address residue (mod 16 bytes, in elements) the kernels peel a short head
+ * and use 16-byte vectors, otherwise they fall back to narrower vectors, with
+ * the same results.  The call is stream-ordered and returns after the step
+ * has finished on the GPU (it synchronises cuda_stream only).  Overflow is
+ * not an error: it returns NEOX_OK with out->overflow = 1.  On
+ * NEOX_ERR_INVALID_ARGUMENT nothing was launched; on NEOX_ERR_CUDA the shard
+ * state is undefined. */
+neox_status neox_shard_step(neox_shard* h, const void* const* grads, int32_t num_grads,
+                            void* params, float lr, void* cuda_stream, neox_step_result* out);
+
+/* Replace the hyperparameters (e.g. the clip 1.0 -> 0.3 change); the current
+ * loss scale and counters are kept (init_scale is ignored here). */
+neox_status neox_shard_set_hparams(neox_shard* h, const neox_hparams* hp);
+
+/* Scaler / step-count state, for checkpoint and resume.  Any pointer may be
+ * NULL.  set_state validates scale > 0 finite, good >= 0, t >= 0. */
+neox_status neox_shard_get_state(const neox_shard* h, float* scale, int32_t* good, int64_t* t);
+neox_status neox_shard_set_state(neox_shard* h, float scale, int32_t good, int64_t t);
+
+/* Free what create allocated (never the caller's arrays).  NULL is a no-op. */
+void neox_shard_destroy(neox_shard* h);
+
+/* Static strings. */
+const char* neox_status_string(neox_status s);
+/* The last error message of this handle ("" if none); NULL handle -> the last
+ * error of a failed create on this thread. */
+const char* neox_last_error(const neox_shard* h);
+
+/* Model-state bytes of numel parameters: 16-bit working weight + 16-bit grad
+ * + FP32 master, m and v = 16 bytes per parameter (host arithmetic only). */
+uint64_t neox_model_state_bytes(uint64_t numel, neox_dtype wdtype, neox_dtype gdtype);
+
+/* Device bytes the handle itself owns (scratch, scalars, segment table). */
+uint64_t neox_shard_scratch_bytes(const neox_shard* h);
+
+/* Per-kernel timing: when enabled, each step records CUDA events around its
+ * two passes on the step's stream and accumulates their durations (read after
+ * the step's own synchronisation, so no extra wait).  `launches` counts every
+ * kernel this handle launched since create, timing on or off. */
+typedef struct {
+    int64_t steps;             /* steps timed since the last reset            */
+    int64_t launches;          /* kernels launched by this handle             */
+    double grad_pass_ms;       /* total of pass 1 (ingest, flag, norm, scaler) */
+    double update_pass_ms;     /* total of pass 2 (AdamW + cast)              */
+    double last_grad_pass_ms;
+    double last_update_pass_ms;
+} neox_profile;
+
+neox_status neox_shard_set_profiling(neox_shard* h, int32_t enable);
+neox_status neox_shard_get_profile(const neox_shard* h, neox_profile* out);
+neox_status neox_shard_reset_profile(neox_shard* h);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NEOX_SHARD_H */

@@ -1,0 +1,130 @@
+"""B200-native per-rank mixed-precision optimizer step over an owned flat shard.
+
+The step (ingest + pre-divide + unscale, overflow flag, global norm, dynamic
+loss scaler, global-norm clip, AdamW on FP32 master/m/v, cast to 16-bit
+working weights) runs in the hand-written CUDA kernels of ``libneoxshard.so``
+(C ABI: ``include/neox_shard.h``).  This package only marshals arguments:
+PyTorch provides device memory and streams.
+
+    from mixed_precision_zero_b200 import NeoxShard, Hparams
+    shard = NeoxShard(master, exp_avg, exp_avg_sq, Hparams(clip_norm=1.0))
+    res = shard.step([grad], params, lr=6e-4)   # res.overflow, res.grad_norm, ...
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+from ._abi import (NEOX_BF16, NEOX_ERR_CUDA, NEOX_ERR_INVALID_ARGUMENT, NEOX_ERR_OUT_OF_MEMORY,  # noqa: F401
+                   NEOX_ERR_UNSUPPORTED, NEOX_FP16, NEOX_OK, NeoxError, lib, neox_hparams,
+                   neox_last_error, neox_model_state_bytes, neox_profile, neox_segment,
+                   neox_shard_create, neox_shard_desc, neox_shard_destroy, neox_shard_get_profile,
+                   neox_shard_get_state, neox_shard_reset_profile, neox_shard_scratch_bytes,
+                   neox_shard_set_hparams, neox_shard_set_profiling, neox_shard_set_state,
+                   neox_shard_step, neox_status_string, neox_step_result)
+
+__all__ = ["NeoxShard", "Hparams", "NeoxError", "neox_shard_create", "neox_shard_step",
+           "neox_shard_destroy", "neox_shard_set_hparams", "neox_shard_get_state",
+           "neox_shard_set_state", "neox_status_string", "neox_last_error", "neox_model_state_bytes"]
+
+
+@dataclass
+class Hparams:
+    beta1: float = 0.9
+    beta2: float = 0.95
+    eps: float = 1e-8
+    clip_norm: float = 1.0
+    predivide: float = 1.0
+    init_scale: float = 65536.0
+    scale_factor: float = 2.0
+    min_scale: float = 1.0
+    scale_window: int = 1000
+
+    def c(self) -> neox_hparams:
+        return neox_hparams(self.beta1, self.beta2, self.eps, self.clip_norm, self.predivide,
+                            self.init_scale, self.scale_factor, self.min_scale, self.scale_window)
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float16:
+        return NEOX_FP16
+    if t.dtype == torch.bfloat16:
+        return NEOX_BF16
+    raise TypeError(f"16-bit tensor must be float16 or bfloat16, got {t.dtype}")
+
+
+class NeoxShard:
+    """One owned flat shard on one GPU: caller-owned FP32 master / exp_avg /
+    exp_avg_sq CUDA tensors of equal length, plus the library handle."""
+
+    def __init__(self, master, exp_avg, exp_avg_sq, hp: Hparams | None = None, *,
+                 wdtype=None, gdtype=None, segments=None, weight_decay: float = 0.0,
+                 max_grads: int = 1, device: int | None = None):
+        import torch
+        hp = hp or Hparams()
+        n = master.numel()
+        for t in (master, exp_avg, exp_avg_sq):
+            if t.dtype != torch.float32 or t.numel() != n or not t.is_contiguous():
+                raise ValueError("master/exp_avg/exp_avg_sq must be contiguous float32 tensors of equal length")
+        self.numel = n
+        self.tensors = (master, exp_avg, exp_avg_sq)  # keep them alive with the handle
+        self.wdtype = NEOX_FP16 if wdtype in (None, torch.float16) else NEOX_BF16
+        self.gdtype = NEOX_FP16 if gdtype in (None, torch.float16) else NEOX_BF16
+        if segments is not None:
+            self._segs = (neox_segment * len(segments))(*[neox_segment(int(o), int(c), float(w))
+                                                          for o, c, w in segments])
+            segp, nsegs = ctypes.cast(self._segs, ctypes.POINTER(neox_segment)), len(segments)
+        else:
+            self._segs, segp, nsegs = None, None, 0
+        desc = neox_shard_desc(n, self.wdtype, self.gdtype, segp, nsegs, float(weight_decay),
+                               master.data_ptr() if n else None, exp_avg.data_ptr() if n else None,
+                               exp_avg_sq.data_ptr() if n else None, int(max_grads))
+        self.device = master.device.index if device is None else device
+        if self.device is None:
+            self.device = torch.cuda.current_device()
+        self.handle = neox_shard_create(desc, hp.c(), self.device)
+
+    def step(self, grads, params, lr: float, stream=None) -> neox_step_result:
+        import torch
+        for g in grads:
+            if g.numel() != self.numel or _dtype_code(g) != self.gdtype or not g.is_contiguous():
+                raise ValueError("each grad must be a contiguous 16-bit tensor of the shard's gradient type and length")
+        if params.numel() != self.numel or _dtype_code(params) != self.wdtype or not params.is_contiguous():
+            raise ValueError("params must be a contiguous 16-bit tensor of the shard's weight type and length")
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device)
+        sp = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+        return neox_shard_step(self.handle, [g.data_ptr() for g in grads], params.data_ptr(), lr, sp)
+
+    def set_hparams(self, hp: Hparams) -> None:
+        neox_shard_set_hparams(self.handle, hp.c())
+
+    def get_state(self):
+        return neox_shard_get_state(self.handle)
+
+    def set_state(self, scale: float, good: int, t: int) -> None:
+        neox_shard_set_state(self.handle, scale, good, t)
+
+    def set_profiling(self, enable: bool) -> None:
+        neox_shard_set_profiling(self.handle, enable)
+
+    def profile(self) -> neox_profile:
+        return neox_shard_get_profile(self.handle)
+
+    def reset_profile(self) -> None:
+        neox_shard_reset_profile(self.handle)
+
+    def scratch_bytes(self) -> int:
+        return neox_shard_scratch_bytes(self.handle)
+
+    def close(self) -> None:
+        if getattr(self, "handle", None):
+            neox_shard_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,180 @@
+"""ctypes declarations of the C ABI in include/neox_shard.h (argument marshalling only).
+
+The functions keep the C names.  Loading fails loudly when the CUDA library
+has not been built: there is no fallback implementation of the step.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libneoxshard.so")
+
+NEOX_OK = 0
+NEOX_ERR_INVALID_ARGUMENT = 1
+NEOX_ERR_CUDA = 2
+NEOX_ERR_OUT_OF_MEMORY = 3
+NEOX_ERR_UNSUPPORTED = 4
+
+NEOX_FP16 = 0
+NEOX_BF16 = 1
+
+
+class neox_segment(ctypes.Structure):
+    _fields_ = [("offset", ctypes.c_uint64), ("numel", ctypes.c_uint64), ("weight_decay", ctypes.c_float)]
+
+
+class neox_hparams(ctypes.Structure):
+    _fields_ = [("beta1", ctypes.c_float), ("beta2", ctypes.c_float), ("eps", ctypes.c_float),
+                ("clip_norm", ctypes.c_float), ("predivide", ctypes.c_float),
+                ("init_scale", ctypes.c_float), ("scale_factor", ctypes.c_float),
+                ("min_scale", ctypes.c_float), ("scale_window", ctypes.c_int32)]
+
+
+class neox_shard_desc(ctypes.Structure):
+    _fields_ = [("numel", ctypes.c_uint64), ("wdtype", ctypes.c_int), ("gdtype", ctypes.c_int),
+                ("segs", ctypes.POINTER(neox_segment)), ("nsegs", ctypes.c_int32),
+                ("default_weight_decay", ctypes.c_float),
+                ("master", ctypes.c_void_p), ("exp_avg", ctypes.c_void_p), ("exp_avg_sq", ctypes.c_void_p),
+                ("max_grads", ctypes.c_int32)]
+
+
+class neox_step_result(ctypes.Structure):
+    _fields_ = [("overflow", ctypes.c_int32), ("grad_norm", ctypes.c_float), ("clip_coef", ctypes.c_float),
+                ("loss_scale", ctypes.c_float), ("loss_scale_next", ctypes.c_float),
+                ("good_steps", ctypes.c_int32), ("applied_steps", ctypes.c_int64)]
+
+    def as_dict(self) -> dict:
+        return {k: getattr(self, k) for k, _ in self._fields_}
+
+
+class neox_profile(ctypes.Structure):
+    _fields_ = [("steps", ctypes.c_int64), ("launches", ctypes.c_int64),
+                ("grad_pass_ms", ctypes.c_double), ("update_pass_ms", ctypes.c_double),
+                ("last_grad_pass_ms", ctypes.c_double), ("last_update_pass_ms", ctypes.c_double)]
+
+
+_lib = None
+_H = ctypes.c_void_p
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"CUDA library {LIB_PATH} is not built; run `python -m mixed_precision_zero_b200.build` "
+                "(there is no CPU fallback for the shard step)")
+        L = ctypes.CDLL(LIB_PATH)
+        S = ctypes.c_int
+        L.neox_shard_create.argtypes = [ctypes.POINTER(neox_shard_desc), ctypes.POINTER(neox_hparams), ctypes.c_int,
+                                        ctypes.POINTER(_H)]
+        L.neox_shard_create.restype = S
+        L.neox_shard_step.argtypes = [_H, ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32, ctypes.c_void_p,
+                                      ctypes.c_float, ctypes.c_void_p, ctypes.POINTER(neox_step_result)]
+        L.neox_shard_step.restype = S
+        L.neox_shard_set_hparams.argtypes = [_H, ctypes.POINTER(neox_hparams)]
+        L.neox_shard_set_hparams.restype = S
+        L.neox_shard_get_state.argtypes = [_H, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int32),
+                                           ctypes.POINTER(ctypes.c_int64)]
+        L.neox_shard_get_state.restype = S
+        L.neox_shard_set_state.argtypes = [_H, ctypes.c_float, ctypes.c_int32, ctypes.c_int64]
+        L.neox_shard_set_state.restype = S
+        L.neox_shard_destroy.argtypes = [_H]
+        L.neox_shard_destroy.restype = None
+        L.neox_status_string.argtypes = [S]
+        L.neox_status_string.restype = ctypes.c_char_p
+        L.neox_last_error.argtypes = [_H]
+        L.neox_last_error.restype = ctypes.c_char_p
+        L.neox_model_state_bytes.argtypes = [ctypes.c_uint64, ctypes.c_int, ctypes.c_int]
+        L.neox_model_state_bytes.restype = ctypes.c_uint64
+        L.neox_shard_scratch_bytes.argtypes = [_H]
+        L.neox_shard_scratch_bytes.restype = ctypes.c_uint64
+        L.neox_shard_set_profiling.argtypes = [_H, ctypes.c_int32]
+        L.neox_shard_set_profiling.restype = S
+        L.neox_shard_get_profile.argtypes = [_H, ctypes.POINTER(neox_profile)]
+        L.neox_shard_get_profile.restype = S
+        L.neox_shard_reset_profile.argtypes = [_H]
+        L.neox_shard_reset_profile.restype = S
+        _lib = L
+    return _lib
+
+
+class NeoxError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{lib().neox_status_string(status).decode()} ({status}): {message}")
+        self.status = status
+
+
+# ---- same-named wrappers -------------------------------------------------------
+
+def neox_shard_create(desc: neox_shard_desc, hp: neox_hparams, device: int) -> int:
+    h = _H()
+    st = lib().neox_shard_create(ctypes.byref(desc), ctypes.byref(hp), device, ctypes.byref(h))
+    if st != NEOX_OK:
+        raise NeoxError(st, lib().neox_last_error(None).decode())
+    return h.value
+
+
+def neox_shard_step(h: int, grad_ptrs, params_ptr: int, lr: float, stream: int) -> neox_step_result:
+    arr = (ctypes.c_void_p * len(grad_ptrs))(*grad_ptrs)
+    res = neox_step_result()
+    st = lib().neox_shard_step(h, arr, len(grad_ptrs), params_ptr, lr, stream, ctypes.byref(res))
+    if st != NEOX_OK:
+        raise NeoxError(st, lib().neox_last_error(h).decode())
+    return res
+
+
+def neox_shard_set_hparams(h: int, hp: neox_hparams) -> None:
+    st = lib().neox_shard_set_hparams(h, ctypes.byref(hp))
+    if st != NEOX_OK:
+        raise NeoxError(st, lib().neox_last_error(h).decode())
+
+
+def neox_shard_get_state(h: int):
+    s, g, t = ctypes.c_float(), ctypes.c_int32(), ctypes.c_int64()
+    st = lib().neox_shard_get_state(h, ctypes.byref(s), ctypes.byref(g), ctypes.byref(t))
+    if st != NEOX_OK:
+        raise NeoxError(st, "get_state")
+    return s.value, g.value, t.value
+
+
+def neox_shard_set_state(h: int, scale: float, good: int, t: int) -> None:
+    st = lib().neox_shard_set_state(h, scale, good, t)
+    if st != NEOX_OK:
+        raise NeoxError(st, lib().neox_last_error(h).decode())
+
+
+def neox_shard_destroy(h: int) -> None:
+    lib().neox_shard_destroy(h)
+
+
+def neox_status_string(status: int) -> str:
+    return lib().neox_status_string(status).decode()
+
+
+def neox_last_error(h: int | None) -> str:
+    return lib().neox_last_error(h).decode()
+
+
+def neox_model_state_bytes(numel: int, wdtype: int = NEOX_FP16, gdtype: int = NEOX_FP16) -> int:
+    return lib().neox_model_state_bytes(numel, wdtype, gdtype)
+
+
+def neox_shard_scratch_bytes(h: int) -> int:
+    return lib().neox_shard_scratch_bytes(h)
+
+
+def neox_shard_set_profiling(h: int, enable: bool) -> None:
+    lib().neox_shard_set_profiling(h, int(enable))
+
+
+def neox_shard_get_profile(h: int) -> neox_profile:
+    p = neox_profile()
+    lib().neox_shard_get_profile(h, ctypes.byref(p))
+    return p
+
+
+def neox_shard_reset_profile(h: int) -> None:
+    lib().neox_shard_reset_profile(h)

@@ -1,0 +1,951 @@
+// neox_shard.cu -- the per-rank mixed-precision optimizer step over an owned
+// flat shard, for NVIDIA B200 (sm_100a).  C ABI in include/neox_shard.h.
+//
+// Pages followed (title, section):
+//  * "GPT-NeoX: how it opened the door to democratised 100B-scale training"
+//    (ainews.cool), "技术深度解析" (technical deep-dive): ZeRO stage 1 -- each
+//    data-parallel rank updates only the optimizer-state shard it owns.
+//  * "OPT: Open Pre-trained Transformer Language Models" (ai-papers.xuzou.cn
+//    summary), "计算设置" (compute setup): FP32 Adam state, FP16 weights,
+//    dynamic loss scaling; "瓶颈" (bottlenecks): 16 bytes/param of state;
+//    "方法适配" (method adaptation): gradient pre-divide, global-norm clip
+//    1.0 / 0.3, loss-scaler reset.
+//  * AdamW (Loshchilov & Hutter) with bias correction: the pages do not
+//    write the update out.
+//
+// Design (HBM-bound, no dense contraction, so no tensor cores):
+//  pass 1  grad_stats_kernel: one streaming read of the K 16-bit gradient
+//          buffers with 16-byte vector loads; pre-divide + FP32 sum +
+//          unscale in registers; non-finite flag; per-thread sum of squares
+//          (FP32 within a vector, FP64 across vectors); warp-shuffle and
+//          shared-memory block reduction to per-block partials.  The last
+//          block to finish (atomic ticket, no spinning) reduces the partials
+//          in a fixed order, so the norm is deterministic, and runs the
+//          loss scaler and the clip coefficient on the device.
+//  pass 2  adam_kernel: one streaming pass over grad (or the FP32 sum),
+//          master, m, v with 16-byte vectors; returns at once when the step
+//          overflowed; AdamW with the clip folded in; writes master, m, v and
+//          the 16-bit working copy with streaming stores.
+// Every FP32 operation of the ingest and of the update uses an explicit
+// round-to-nearest intrinsic (no contraction), in the same order as the plain
+// definition, so for equal clip coefficients the results are bit-exact with
+// a sequential FP32 evaluation.
+
+#include "neox_shard.h"
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+
+namespace {
+
+constexpr int kMaxGrads = 64;
+constexpr int kThreads1 = 512;   // pass-1 block
+constexpr int kThreads3 = 256;   // pass-2 block
+constexpr int kMaxBlocksPerSm = 32;
+
+struct GradPtrs {
+    const uint16_t* p[kMaxGrads];
+};
+
+// Device-resident scalars of one shard (64 bytes).  `scale`, `good`, `t` are
+// the scaler / step state; the rest describe the most recent step.
+struct __align__(64) DevScalars {
+    double sumsq;          // sum of squared unscaled grads of the last step
+    float scale;           // S the next step's grads carry
+    int32_t good;          // consecutive applied steps
+    long long t;           // applied steps
+    int32_t overflow;      // last step overflowed
+    float coef;            // clip coefficient of the last step
+    float scale_used;      // S the last step's grads carried
+    float norm;            // pre-clip norm of the last step (+inf on overflow)
+    unsigned int blocks_done;  // pass-1 ticket counter, back to 0 after each step
+    int32_t pad_[5];
+};
+static_assert(sizeof(DevScalars) == 64, "DevScalars is one 64-byte block");
+
+// Which elements use vectors: [0, head) scalar, [head, head + nvec*VEC)
+// vectors of VEC, [tail0, n) scalar.
+struct Layout {
+    unsigned long long n, head, nvec, tail0;
+};
+
+struct ScalerArgs {
+    double post;          // K / predivide
+    float inv_pre;        // fl32(1 / predivide)
+    float clip;           // <= 0: off
+    float factor, min_scale;
+    int32_t window;
+};
+
+struct AdamArgs {
+    float lr, b1, b2, omb1, omb2, eps;
+    float step_size;      // fl32(lr / bc1) for t+1
+    float bcs;            // fl32(sqrt(bc2)) for t+1
+    float inv_pre;
+    double post;
+};
+
+// ---------------------------------------------------------------- 16-bit types
+struct F16 {
+    static __device__ __forceinline__ float dec(uint16_t h) { return __half2float(__ushort_as_half(h)); }
+    static __device__ __forceinline__ uint16_t enc(float f) { return __half_as_ushort(__float2half_rn(f)); }
+    static __device__ __forceinline__ uint32_t enc2(float lo, float hi) {
+        __half2 h = __floats2half2_rn(lo, hi);
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+};
+struct BF16 {
+    static __device__ __forceinline__ float dec(uint16_t h) { return __uint_as_float(uint32_t(h) << 16); }
+    static __device__ __forceinline__ uint16_t enc(float f) { return __bfloat16_as_ushort(__float2bfloat16_rn(f)); }
+    static __device__ __forceinline__ uint32_t enc2(float lo, float hi) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+};
+
+// ---------------------------------------------------------------- vector I/O
+// VEC 16-bit values starting at p (aligned to 2*VEC bytes), read-only data.
+template <int VEC>
+__device__ __forceinline__ void ld16(const uint16_t* p, uint16_t (&o)[VEC]) {
+    if constexpr (VEC == 8) {
+        uint4 r = __ldcs(reinterpret_cast<const uint4*>(p));
+        uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int i = 0; i < 4; i++) { o[2 * i] = uint16_t(w[i]); o[2 * i + 1] = uint16_t(w[i] >> 16); }
+    } else if constexpr (VEC == 4) {
+        uint2 r = __ldcs(reinterpret_cast<const uint2*>(p));
+        o[0] = uint16_t(r.x); o[1] = uint16_t(r.x >> 16); o[2] = uint16_t(r.y); o[3] = uint16_t(r.y >> 16);
+    } else if constexpr (VEC == 2) {
+        uint32_t r = __ldcs(reinterpret_cast<const unsigned int*>(p));
+        o[0] = uint16_t(r); o[1] = uint16_t(r >> 16);
+    } else {
+        o[0] = __ldcs(reinterpret_cast<const unsigned short*>(p));
+    }
+}
+
+template <class W, int VEC>
+__device__ __forceinline__ void st16(uint16_t* p, const float (&x)[VEC]) {
+    if constexpr (VEC == 8) {
+        uint4 r = make_uint4(W::enc2(x[0], x[1]), W::enc2(x[2], x[3]), W::enc2(x[4], x[5]), W::enc2(x[6], x[7]));
+        __stcs(reinterpret_cast<uint4*>(p), r);
+    } else if constexpr (VEC == 4) {
+        uint2 r = make_uint2(W::enc2(x[0], x[1]), W::enc2(x[2], x[3]));
+        __stcs(reinterpret_cast<uint2*>(p), r);
+    } else if constexpr (VEC == 2) {
+        __stcs(reinterpret_cast<unsigned int*>(p), W::enc2(x[0], x[1]));
+    } else {
+        __stcs(reinterpret_cast<unsigned short*>(p), W::enc(x[0]));
+    }
+}
+
+// VEC FP32 values at p (16-byte aligned when VEC >= 4).
+template <int VEC>
+__device__ __forceinline__ void ld32(const float* p, float (&o)[VEC]) {
+    if constexpr (VEC >= 4) {
+#pragma unroll
+        for (int q = 0; q < VEC / 4; q++) {
+            float4 r = __ldcs(reinterpret_cast<const float4*>(p) + q);
+            o[4 * q] = r.x; o[4 * q + 1] = r.y; o[4 * q + 2] = r.z; o[4 * q + 3] = r.w;
+        }
+    } else if constexpr (VEC == 2) {
+        float2 r = __ldcs(reinterpret_cast<const float2*>(p));
+        o[0] = r.x; o[1] = r.y;
+    } else {
+        o[0] = __ldcs(p);
+    }
+}
+
+template <int VEC>
+__device__ __forceinline__ void st32(float* p, const float (&x)[VEC]) {
+    if constexpr (VEC >= 4) {
+#pragma unroll
+        for (int q = 0; q < VEC / 4; q++)
+            __stcs(reinterpret_cast<float4*>(p) + q, make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]));
+    } else if constexpr (VEC == 2) {
+        __stcs(reinterpret_cast<float2*>(p), make_float2(x[0], x[1]));
+    } else {
+        __stcs(p, x[0]);
+    }
+}
+
+__device__ __forceinline__ bool not_finite(float x) {
+    return (__float_as_uint(x) & 0x7f800000u) == 0x7f800000u;
+}
+
+// Unscaled gradients of VEC consecutive elements from global index i:
+// a = sum_k fl32(g_k * inv_pre) in buffer order (starting from +0, as a
+// sequential sum does), then fl32(a * inv_us).
+template <class G, int VEC>
+__device__ __forceinline__ void ingest(const GradPtrs& gp, int K, unsigned long long i,
+                                       float inv_pre, float inv_us, float (&g)[VEC]) {
+#pragma unroll
+    for (int e = 0; e < VEC; e++) g[e] = 0.0f;
+    for (int k = 0; k < K; k++) {
+        uint16_t h[VEC];
+        ld16<VEC>(gp.p[k] + i, h);
+#pragma unroll
+        for (int e = 0; e < VEC; e++) g[e] = __fadd_rn(g[e], __fmul_rn(G::dec(h[e]), inv_pre));
+    }
+#pragma unroll
+    for (int e = 0; e < VEC; e++) g[e] = __fmul_rn(g[e], inv_us);
+}
+
+__device__ __forceinline__ float unscale_factor(double post, float scale) {
+    return (float)(1.0 / (post * (double)scale));
+}
+
+// Sum of squares of a vector: FP32 within the vector, recomputed in FP64 in
+// the (degenerate) case that a finite element squares past FP32's range.
+template <int VEC>
+__device__ __forceinline__ double vec_sumsq(const float (&g)[VEC], int& bad) {
+    float q = 0.0f;
+    int vb = 0;
+#pragma unroll
+    for (int e = 0; e < VEC; e++) {
+        vb |= not_finite(g[e]);
+        q = __fmaf_rn(g[e], g[e], q);
+    }
+    bad |= vb;
+    if (!vb && not_finite(q)) {
+        double d = 0.0;
+#pragma unroll
+        for (int e = 0; e < VEC; e++) d += (double)g[e] * (double)g[e];
+        return d;
+    }
+    return (double)q;
+}
+
+// Block-wide reduction of (double, int-or) with a fixed shape.
+template <int THREADS>
+__device__ __forceinline__ void block_reduce(double& s, int& bad, double* sh_s, int* sh_b) {
+    const unsigned full = 0xffffffffu;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        s += __shfl_down_sync(full, s, off);
+        bad |= __shfl_down_sync(full, bad, off);
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) { sh_s[warp] = s; sh_b[warp] = bad; }
+    __syncthreads();
+    if (warp == 0) {
+        constexpr int NW = THREADS / 32;
+        s = lane < NW ? sh_s[lane] : 0.0;
+        bad = lane < NW ? sh_b[lane] : 0;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            s += __shfl_down_sync(full, s, off);
+            bad |= __shfl_down_sync(full, bad, off);
+        }
+    }
+}
+
+// ---------------------------------------------------------------- pass 1
+template <class G, int VEC, bool WRITE_ACC>
+__global__ void __launch_bounds__(kThreads1)
+grad_stats_kernel(GradPtrs gp, int K, Layout L, ScalerArgs sa, float* __restrict__ acc,
+                  double* __restrict__ part_s, int* __restrict__ part_b, DevScalars* __restrict__ sc) {
+    __shared__ double sh_s[kThreads1 / 32];
+    __shared__ int sh_b[kThreads1 / 32];
+    __shared__ bool is_last;
+
+    const float inv_us = unscale_factor(sa.post, sc->scale);
+    double s = 0.0;
+    int bad = 0;
+
+    const unsigned long long stride = (unsigned long long)gridDim.x * kThreads1;
+    for (unsigned long long v = (unsigned long long)blockIdx.x * kThreads1 + threadIdx.x; v < L.nvec; v += stride) {
+        const unsigned long long i = L.head + v * VEC;
+        float g[VEC];
+        ingest<G, VEC>(gp, K, i, sa.inv_pre, inv_us, g);
+        s += vec_sumsq<VEC>(g, bad);
+        if constexpr (WRITE_ACC) st32<VEC>(acc + i, g);
+    }
+    if (blockIdx.x == 0) {  // peeled head and ragged tail, one element per thread
+        const unsigned long long extra = L.head + (L.n - L.tail0);
+        for (unsigned long long j = threadIdx.x; j < extra; j += kThreads1) {
+            const unsigned long long i = j < L.head ? j : L.tail0 + (j - L.head);
+            float g[1];
+            ingest<G, 1>(gp, K, i, sa.inv_pre, inv_us, g);
+            s += vec_sumsq<1>(g, bad);
+            if constexpr (WRITE_ACC) acc[i] = g[0];
+        }
+    }
+
+    block_reduce<kThreads1>(s, bad, sh_s, sh_b);
+    if (threadIdx.x == 0) {
+        part_s[blockIdx.x] = s;
+        part_b[blockIdx.x] = bad;
+        __threadfence();
+        const unsigned ticket = atomicAdd(&sc->blocks_done, 1u);
+        is_last = (ticket == gridDim.x - 1);
+    }
+    __syncthreads();
+    if (!is_last) return;
+
+    // Last block: every other block's partial is visible (each fenced before
+    // taking its ticket).  Reduce them in a fixed order.
+    __threadfence();
+    s = 0.0;
+    bad = 0;
+    for (unsigned j = threadIdx.x; j < gridDim.x; j += kThreads1) {
+        s += __ldcg(part_s + j);
+        bad |= __ldcg(part_b + j);
+    }
+    __syncthreads();
+    block_reduce<kThreads1>(s, bad, sh_s, sh_b);
+    if (threadIdx.x != 0) return;
+
+    // Scalar decisions of the step.
+    int overflow = bad != 0;
+    const double norm = sqrt(s);
+    if (!overflow && !isfinite(norm)) overflow = 1;
+    float S = sc->scale;
+    int good = sc->good;
+    long long t = sc->t;
+    sc->scale_used = S;
+    sc->sumsq = s;
+    sc->overflow = overflow;
+    if (overflow) {
+        const float d = S / sa.factor;
+        S = d > sa.min_scale ? d : sa.min_scale;
+        good = 0;
+        sc->coef = 0.0f;
+        sc->norm = __int_as_float(0x7f800000);
+    } else {
+        good += 1;
+        if (good >= sa.window) {
+            const float u = S * sa.factor;
+            if (!not_finite(u)) S = u;
+            good = 0;
+        }
+        t += 1;
+        float c = 1.0f;
+        if (sa.clip > 0.0f) {
+            const double cd = (double)sa.clip / (norm + 1e-6);
+            if (cd < 1.0) c = (float)cd;
+        }
+        sc->coef = c;
+        sc->norm = (float)norm;
+    }
+    sc->scale = S;
+    sc->good = good;
+    sc->t = t;
+    sc->blocks_done = 0;
+}
+
+// ---------------------------------------------------------------- pass 2
+struct SegCursor {
+    int seg;
+    unsigned long long end;
+    float keep;  // fl32(1 - fl32(lr * wd)) of segment `seg`
+};
+
+__device__ __forceinline__ void seg_seek(SegCursor& c, unsigned long long i, const unsigned long long* seg_end,
+                                         const float* seg_wd, int nsegs, float lr) {
+    // first segment whose end is > i, searching from the current one
+    int lo = c.seg, hi = nsegs - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(seg_end + mid) > i) hi = mid; else lo = mid + 1;
+    }
+    c.seg = lo;
+    c.end = __ldg(seg_end + lo);
+    c.keep = __fsub_rn(1.0f, __fmul_rn(lr, __ldg(seg_wd + lo)));
+}
+
+template <int VEC>
+__device__ __forceinline__ void adam_vec(const float (&g)[VEC], const float (&keep)[VEC], float c,
+                                         const AdamArgs& a, float (&p)[VEC], float (&m)[VEC], float (&v)[VEC]) {
+#pragma unroll
+    for (int e = 0; e < VEC; e++) {
+        const float gh = __fmul_rn(g[e], c);
+        const float mj = __fadd_rn(__fmul_rn(a.b1, m[e]), __fmul_rn(a.omb1, gh));
+        const float gg = __fmul_rn(a.omb2, gh);
+        const float vj = __fadd_rn(__fmul_rn(a.b2, v[e]), __fmul_rn(gg, gh));
+        const float den = __fadd_rn(__fdiv_rn(__fsqrt_rn(vj), a.bcs), a.eps);
+        float pj = __fmul_rn(p[e], keep[e]);
+        const float upd = __fdiv_rn(mj, den);
+        pj = __fsub_rn(pj, __fmul_rn(a.step_size, upd));
+        m[e] = mj;
+        v[e] = vj;
+        p[e] = pj;
+    }
+}
+
+template <class G, class W, int VEC, bool READ_ACC>
+__global__ void __launch_bounds__(kThreads3)
+adam_kernel(GradPtrs gp, int K, const float* __restrict__ acc, Layout L, AdamArgs a,
+            float* __restrict__ master, float* __restrict__ m, float* __restrict__ v, uint16_t* __restrict__ w,
+            const unsigned long long* __restrict__ seg_end, const float* __restrict__ seg_wd, int nsegs,
+            const DevScalars* __restrict__ sc) {
+    if (sc->overflow) return;  // skipped step: nothing is written
+    const float c = sc->coef;
+    const float inv_us = unscale_factor(a.post, sc->scale_used);
+
+    const unsigned long long stride = (unsigned long long)gridDim.x * kThreads3;
+    unsigned long long v0 = (unsigned long long)blockIdx.x * kThreads3 + threadIdx.x;
+    SegCursor cur{0, 0ull, 1.0f};
+    if (v0 < L.nvec) seg_seek(cur, L.head + v0 * VEC, seg_end, seg_wd, nsegs, a.lr);
+
+    for (unsigned long long vi = v0; vi < L.nvec; vi += stride) {
+        const unsigned long long i = L.head + vi * VEC;
+        float g[VEC], p[VEC], mm[VEC], vv[VEC], keep[VEC];
+        if constexpr (READ_ACC) ld32<VEC>(acc + i, g);
+        else ingest<G, VEC>(gp, K, i, a.inv_pre, inv_us, g);
+        ld32<VEC>(master + i, p);
+        ld32<VEC>(m + i, mm);
+        ld32<VEC>(v + i, vv);
+        if (i >= cur.end) seg_seek(cur, i, seg_end, seg_wd, nsegs, a.lr);
+        if (i + VEC <= cur.end) {
+#pragma unroll
+            for (int e = 0; e < VEC; e++) keep[e] = cur.keep;
+        } else {
+#pragma unroll
+            for (int e = 0; e < VEC; e++) {
+                if (i + e >= cur.end) seg_seek(cur, i + e, seg_end, seg_wd, nsegs, a.lr);
+                keep[e] = cur.keep;
+            }
+        }
+        adam_vec<VEC>(g, keep, c, a, p, mm, vv);
+        st32<VEC>(master + i, p);
+        st32<VEC>(m + i, mm);
+        st32<VEC>(v + i, vv);
+        st16<W, VEC>(w + i, p);
+    }
+    if (blockIdx.x == 0) {
+        const unsigned long long extra = L.head + (L.n - L.tail0);
+        for (unsigned long long j = threadIdx.x; j < extra; j += kThreads3) {
+            const unsigned long long i = j < L.head ? j : L.tail0 + (j - L.head);
+            float g[1], p[1] = {master[i]}, mm[1] = {m[i]}, vv[1] = {v[i]}, keep[1];
+            if constexpr (READ_ACC) g[0] = acc[i];
+            else ingest<G, 1>(gp, K, i, a.inv_pre, inv_us, g);
+            SegCursor c1{0, 0ull, 1.0f};
+            seg_seek(c1, i, seg_end, seg_wd, nsegs, a.lr);
+            keep[0] = c1.keep;
+            adam_vec<1>(g, keep, c, a, p, mm, vv);
+            master[i] = p[0];
+            m[i] = mm[0];
+            v[i] = vv[0];
+            w[i] = W::enc(p[0]);
+        }
+    }
+}
+
+}  // namespace
+
+// ====================================================================== host
+
+struct neox_shard {
+    int device = 0;
+    int sm_count = 0;
+    unsigned long long numel = 0;
+    neox_dtype wdtype = NEOX_FP16, gdtype = NEOX_FP16;
+    float* master = nullptr;
+    float* m = nullptr;
+    float* v = nullptr;
+    neox_hparams hp{};
+    int max_grads = 1;
+    // mirrors of the device scaler state (refreshed after every step)
+    float scale = 1.0f;
+    int32_t good = 0;
+    long long t = 0;
+    // owned device memory
+    DevScalars* d_sc = nullptr;
+    double* d_part_s = nullptr;
+    int* d_part_b = nullptr;
+    int max_parts = 0;
+    unsigned long long* d_seg_end = nullptr;
+    float* d_seg_wd = nullptr;
+    int nsegs = 0;
+    float* d_acc = nullptr;  // FP32 sum of K >= 5 buffers (numel + 4 floats)
+    DevScalars* h_sc = nullptr;  // pinned result slot
+    unsigned long long owned_bytes = 0;
+    // profiling
+    bool profiling = false;
+    cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};
+    neox_profile prof{};
+    std::string last_error;
+};
+
+namespace {
+
+thread_local std::string g_create_error;
+
+struct DeviceGuard {
+    int prev = -1;
+    bool ok = true;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+        if (prev != dev) ok = cudaSetDevice(dev) == cudaSuccess;
+    }
+    ~DeviceGuard() {
+        int cur = -1;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+};
+
+neox_status fail(neox_shard* h, neox_status st, const std::string& msg) {
+    if (h) h->last_error = msg; else g_create_error = msg;
+    return st;
+}
+
+neox_status cuda_fail(neox_shard* h, cudaError_t e, const char* what) {
+    std::string msg = std::string(what) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")";
+    return fail(h, e == cudaErrorMemoryAllocation ? NEOX_ERR_OUT_OF_MEMORY : NEOX_ERR_CUDA, msg);
+}
+
+bool finite(float x) { return std::isfinite(x); }
+
+const char* check_hparams(const neox_hparams* hp) {
+    if (!hp) return "hparams is NULL";
+    if (!(hp->beta1 >= 0.0f && hp->beta1 < 1.0f)) return "beta1 must be in [0, 1)";
+    if (!(hp->beta2 >= 0.0f && hp->beta2 < 1.0f)) return "beta2 must be in [0, 1)";
+    if (!(hp->eps >= 0.0f) || !finite(hp->eps)) return "eps must be finite and >= 0";
+    if (!finite(hp->clip_norm)) return "clip_norm must be finite";
+    if (!(hp->predivide > 0.0f) || !finite(hp->predivide)) return "predivide must be finite and > 0";
+    if (!(hp->init_scale > 0.0f) || !finite(hp->init_scale)) return "init_scale must be finite and > 0";
+    if (!(hp->scale_factor >= 1.0f) || !finite(hp->scale_factor)) return "scale_factor must be finite and >= 1";
+    if (!(hp->min_scale >= 0.0f) || !finite(hp->min_scale)) return "min_scale must be finite and >= 0";
+    if (hp->scale_window < 1) return "scale_window must be >= 1";
+    return nullptr;
+}
+
+int elem_size(neox_dtype) { return 2; }
+
+// Choose the widest vector (8, 4, 2, 1 elements) and a head h < VEC such that
+// every 16-bit array is 2*VEC-byte aligned and every FP32 array 16-byte (VEC
+// >= 4) or 4*VEC-byte aligned at element h.
+Layout choose_layout(unsigned long long n, const uintptr_t* a16, int n16, const uintptr_t* a32, int n32, int& vec_out) {
+    for (int vec = 8; vec >= 1; vec >>= 1) {
+        const uintptr_t al16 = 2u * vec;
+        const uintptr_t al32 = vec >= 4 ? 16u : 4u * vec;
+        for (int h = 0; h < vec; h++) {
+            bool ok = true;
+            for (int i = 0; i < n16 && ok; i++) ok = ((a16[i] + 2u * h) % al16) == 0;
+            for (int i = 0; i < n32 && ok; i++) ok = ((a32[i] + 4u * h) % al32) == 0;
+            if (!ok) continue;
+            Layout L;
+            L.n = n;
+            L.head = (unsigned long long)h < n ? h : n;
+            L.nvec = (n - L.head) / vec;
+            L.tail0 = L.head + L.nvec * vec;
+            vec_out = vec;
+            return L;
+        }
+    }
+    vec_out = 1;  // unreachable: VEC = 1 always fits
+    return Layout{n, 0, n, n};
+}
+
+// Resident blocks per SM of one kernel instantiation (queried once per
+// instantiation and device; B200 parts are uniform, so the first answer holds).
+template <class K>
+int occupancy(K kernel, int threads) {
+    static int cached = 0;
+    if (cached == 0) {
+        int occ = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, threads, 0) != cudaSuccess || occ < 1) occ = 1;
+        cached = occ;
+    }
+    return cached;
+}
+
+template <class K>
+int grid_for(K kernel, int threads, unsigned long long work_items, int sm_count, int cap) {
+    const int occ = occupancy(kernel, threads);
+    unsigned long long want = (work_items + threads - 1) / threads;
+    unsigned long long full = (unsigned long long)sm_count * (unsigned long long)occ;
+    unsigned long long g = want < full ? want : full;
+    if (g < 1) g = 1;
+    if (g > (unsigned long long)cap) g = cap;
+    return (int)g;
+}
+
+template <class G, int VEC, bool ACC>
+cudaError_t launch_pass1(neox_shard* h, const GradPtrs& gp, int K, const Layout& L, const ScalerArgs& sa,
+                         float* acc, cudaStream_t st) {
+    auto kern = grad_stats_kernel<G, VEC, ACC>;
+    const int grid = grid_for(kern, kThreads1, L.nvec, h->sm_count, h->max_parts);
+    kern<<<grid, kThreads1, 0, st>>>(gp, K, L, sa, acc, h->d_part_s, h->d_part_b, h->d_sc);
+    return cudaGetLastError();
+}
+
+template <class G, class W, int VEC, bool ACC>
+cudaError_t launch_pass2(neox_shard* h, const GradPtrs& gp, int K, const float* acc, const Layout& L,
+                         const AdamArgs& a, uint16_t* w, cudaStream_t st) {
+    auto kern = adam_kernel<G, W, VEC, ACC>;
+    const int grid = grid_for(kern, kThreads3, L.nvec, h->sm_count, 1 << 20);
+    kern<<<grid, kThreads3, 0, st>>>(gp, K, acc, L, a, h->master, h->m, h->v, w, h->d_seg_end, h->d_seg_wd,
+                                     h->nsegs, h->d_sc);
+    return cudaGetLastError();
+}
+
+template <class G, int VEC>
+cudaError_t dispatch1(neox_shard* h, const GradPtrs& gp, int K, const Layout& L, const ScalerArgs& sa,
+                      float* acc, cudaStream_t st) {
+    return acc ? launch_pass1<G, VEC, true>(h, gp, K, L, sa, acc, st)
+               : launch_pass1<G, VEC, false>(h, gp, K, L, sa, acc, st);
+}
+
+template <class G>
+cudaError_t dispatch1v(neox_shard* h, int vec, const GradPtrs& gp, int K, const Layout& L, const ScalerArgs& sa,
+                       float* acc, cudaStream_t st) {
+    switch (vec) {
+        case 8: return dispatch1<G, 8>(h, gp, K, L, sa, acc, st);
+        case 4: return dispatch1<G, 4>(h, gp, K, L, sa, acc, st);
+        case 2: return dispatch1<G, 2>(h, gp, K, L, sa, acc, st);
+        default: return dispatch1<G, 1>(h, gp, K, L, sa, acc, st);
+    }
+}
+
+template <class G, class W, int VEC>
+cudaError_t dispatch2(neox_shard* h, const GradPtrs& gp, int K, const float* acc, const Layout& L,
+                      const AdamArgs& a, uint16_t* w, cudaStream_t st) {
+    return acc ? launch_pass2<G, W, VEC, true>(h, gp, K, acc, L, a, w, st)
+               : launch_pass2<G, W, VEC, false>(h, gp, K, acc, L, a, w, st);
+}
+
+template <class G, class W>
+cudaError_t dispatch2v(neox_shard* h, int vec, const GradPtrs& gp, int K, const float* acc, const Layout& L,
+                       const AdamArgs& a, uint16_t* w, cudaStream_t st) {
+    switch (vec) {
+        case 8: return dispatch2<G, W, 8>(h, gp, K, acc, L, a, w, st);
+        case 4: return dispatch2<G, W, 4>(h, gp, K, acc, L, a, w, st);
+        case 2: return dispatch2<G, W, 2>(h, gp, K, acc, L, a, w, st);
+        default: return dispatch2<G, W, 1>(h, gp, K, acc, L, a, w, st);
+    }
+}
+
+void free_all(neox_shard* h) {
+    if (h->d_sc) cudaFree(h->d_sc);
+    if (h->d_part_s) cudaFree(h->d_part_s);
+    if (h->d_part_b) cudaFree(h->d_part_b);
+    if (h->d_seg_end) cudaFree(h->d_seg_end);
+    if (h->d_seg_wd) cudaFree(h->d_seg_wd);
+    if (h->d_acc) cudaFree(h->d_acc);
+    if (h->h_sc) cudaFreeHost(h->h_sc);
+    for (auto& e : h->ev)
+        if (e) cudaEventDestroy(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* neox_status_string(neox_status s) {
+    switch (s) {
+        case NEOX_OK: return "ok";
+        case NEOX_ERR_INVALID_ARGUMENT: return "invalid argument";
+        case NEOX_ERR_CUDA: return "CUDA error";
+        case NEOX_ERR_OUT_OF_MEMORY: return "out of memory";
+        case NEOX_ERR_UNSUPPORTED: return "unsupported";
+    }
+    return "unknown status";
+}
+
+const char* neox_last_error(const neox_shard* h) {
+    return h ? h->last_error.c_str() : g_create_error.c_str();
+}
+
+uint64_t neox_model_state_bytes(uint64_t numel, neox_dtype wdtype, neox_dtype gdtype) {
+    return numel * (uint64_t)(elem_size(wdtype) + elem_size(gdtype) + 3 * (int)sizeof(float));
+}
+
+uint64_t neox_shard_scratch_bytes(const neox_shard* h) { return h ? h->owned_bytes : 0; }
+
+neox_status neox_shard_create(const neox_shard_desc* d, const neox_hparams* hp, int device, neox_shard** out) {
+    g_create_error.clear();
+    if (!out) return fail(nullptr, NEOX_ERR_INVALID_ARGUMENT, "out is NULL");
+    if (!d) return fail(nullptr, NEOX_ERR_INVALID_ARGUMENT, "desc is NULL");
+    if (const char* why = check_hparams(hp)) return fail(nullptr, NEOX_ERR_INVALID_ARGUMENT, why);
+    if ((d->wdtype != NEOX_FP16 && d->wdtype != NEOX_BF16) || (d->gdtype != NEOX_FP16 && d->gdtype != NEOX_BF16))
+        return fail(nullptr, NEOX_ERR_INVALID_ARGUMENT, "dtype must be NEOX_FP16 or NEOX_BF16");
+    if (d->max_grads < 0 || d->max_grads > kMaxGrads)
+        return fail(nullptr, NEOX_ERR_INVALID_ARGUMENT, "max_grads must be in [0, 64]");
+    if (d->numel > 0) {
+        if (!d->master || !d->exp_avg || !d->exp_avg_sq)
+            return fail(nullptr, NEOX_ERR_INVALID_ARGUMENT, "master/exp_avg/exp_avg_sq must be non-NULL");
+        if (((uintptr_t)d->master | (uintptr_t)d->exp_avg | (uintptr_t)d->exp_avg_sq) & 3u)
+            return fail(nullptr, NEOX_ERR_INVALID_ARGUMENT, "FP32 state arrays must be 4-byte aligned");
+    }
+    if (!finite(d->default_weight_decay)) return fail(nullptr, NEOX_ERR_INVALID_ARGUMENT, "weight decay must be finite");
+    // segment table -> (end, wd) arrays
+    int nsegs = 1;
+    unsigned long long* ends = nullptr;
+    float* wds = nullptr;
+    if (d->segs) {
+        if (d->nsegs < 1) return fail(nullptr, NEOX_ERR_INVALID_ARGUMENT, "nsegs must be >= 1 with a table");
+        nsegs = d->nsegs;
+        unsigned long long pos = 0;
+        for (int i = 0; i < nsegs; i++) {
+            const neox_segment& s = d->segs[i];
+            if (s.offset != pos || s.numel == 0)
+                return fail(nullptr, NEOX_ERR_INVALID_ARGUMENT,
+                            "segments must be sorted, non-empty and tile [0, numel) (segment " + std::to_string(i) + ")");
+            if (!finite(s.weight_decay))
+                return fail(nullptr, NEOX_ERR_INVALID_ARGUMENT, "segment weight decay must be finite");
+            pos += s.numel;
+        }
+        if (pos != d->numel) return fail(nullptr, NEOX_ERR_INVALID_ARGUMENT, "segments do not cover numel");
+    }
+    ends = new (std::nothrow) unsigned long long[nsegs];
+    wds = new (std::nothrow) float[nsegs];
+    if (!ends || !wds) {
+        delete[] ends;
+        delete[] wds;
+        return fail(nullptr, NEOX_ERR_OUT_OF_MEMORY, "host allocation failed");
+    }
+    if (d->segs) {
+        for (int i = 0; i < nsegs; i++) { ends[i] = d->segs[i].offset + d->segs[i].numel; wds[i] = d->segs[i].weight_decay; }
+    } else {
+        ends[0] = d->numel;
+        wds[0] = d->default_weight_decay;
+    }
+
+    auto* h = new (std::nothrow) neox_shard();
+    if (!h) { delete[] ends; delete[] wds; return fail(nullptr, NEOX_ERR_OUT_OF_MEMORY, "host allocation failed"); }
+    h->device = device;
+    h->numel = d->numel;
+    h->wdtype = d->wdtype;
+    h->gdtype = d->gdtype;
+    h->master = d->master;
+    h->m = d->exp_avg;
+    h->v = d->exp_avg_sq;
+    h->hp = *hp;
+    h->max_grads = d->max_grads < 1 ? 1 : d->max_grads;
+    h->scale = hp->init_scale;
+    h->nsegs = nsegs;
+
+    neox_status st = NEOX_OK;
+    cudaError_t e;
+    {
+        int ndev = 0;
+        if ((e = cudaGetDeviceCount(&ndev)) != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaGetDeviceCount"); goto done; }
+        if (device < 0 || device >= ndev) { st = fail(nullptr, NEOX_ERR_INVALID_ARGUMENT, "no such CUDA device"); goto done; }
+        DeviceGuard g(device);
+        if (!g.ok) { st = fail(nullptr, NEOX_ERR_CUDA, "cudaSetDevice failed"); goto done; }
+        cudaDeviceProp prop;
+        if ((e = cudaGetDeviceProperties(&prop, device)) != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaGetDeviceProperties"); goto done; }
+        if (prop.major != 10) { st = fail(nullptr, NEOX_ERR_UNSUPPORTED, "this library is built for sm_100a (B200)"); goto done; }
+        h->sm_count = prop.multiProcessorCount;
+        h->max_parts = h->sm_count * kMaxBlocksPerSm;
+        size_t bytes;
+        if ((e = cudaMalloc(&h->d_sc, sizeof(DevScalars))) != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMalloc scalars"); goto done; }
+        bytes = sizeof(DevScalars);
+        if ((e = cudaMalloc(&h->d_part_s, sizeof(double) * h->max_parts)) != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMalloc partials"); goto done; }
+        if ((e = cudaMalloc(&h->d_part_b, sizeof(int) * h->max_parts)) != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMalloc partials"); goto done; }
+        bytes += (sizeof(double) + sizeof(int)) * h->max_parts;
+        if ((e = cudaMalloc(&h->d_seg_end, sizeof(unsigned long long) * nsegs)) != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMalloc segments"); goto done; }
+        if ((e = cudaMalloc(&h->d_seg_wd, sizeof(float) * nsegs)) != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMalloc segments"); goto done; }
+        bytes += (sizeof(unsigned long long) + sizeof(float)) * nsegs;
+        if (h->max_grads >= 5 && h->numel > 0) {
+            if ((e = cudaMalloc(&h->d_acc, sizeof(float) * (h->numel + 4))) != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMalloc accumulation buffer"); goto done; }
+            bytes += sizeof(float) * (h->numel + 4);
+        }
+        h->owned_bytes = bytes;
+        if ((e = cudaMallocHost(&h->h_sc, sizeof(DevScalars))) != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMallocHost"); goto done; }
+        for (auto& ev : h->ev)
+            if ((e = cudaEventCreate(&ev)) != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaEventCreate"); goto done; }
+        if ((e = cudaMemcpy(h->d_seg_end, ends, sizeof(unsigned long long) * nsegs, cudaMemcpyHostToDevice)) != cudaSuccess ||
+            (e = cudaMemcpy(h->d_seg_wd, wds, sizeof(float) * nsegs, cudaMemcpyHostToDevice)) != cudaSuccess) {
+            st = cuda_fail(nullptr, e, "cudaMemcpy segments");
+            goto done;
+        }
+        DevScalars init{};
+        init.scale = hp->init_scale;
+        init.scale_used = hp->init_scale;
+        if ((e = cudaMemcpy(h->d_sc, &init, sizeof(init), cudaMemcpyHostToDevice)) != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMemcpy scalars"); goto done; }
+    }
+done:
+    delete[] ends;
+    delete[] wds;
+    if (st != NEOX_OK) {
+        DeviceGuard g(device);
+        free_all(h);
+        delete h;
+        return st;
+    }
+    *out = h;
+    return NEOX_OK;
+}
+
+void neox_shard_destroy(neox_shard* h) {
+    if (!h) return;
+    {
+        DeviceGuard g(h->device);
+        free_all(h);
+    }
+    delete h;
+}
+
+neox_status neox_shard_set_hparams(neox_shard* h, const neox_hparams* hp) {
+    if (!h) return NEOX_ERR_INVALID_ARGUMENT;
+    if (const char* why = check_hparams(hp)) return fail(h, NEOX_ERR_INVALID_ARGUMENT, why);
+    h->hp = *hp;
+    return NEOX_OK;
+}
+
+neox_status neox_shard_get_state(const neox_shard* h, float* scale, int32_t* good, int64_t* t) {
+    if (!h) return NEOX_ERR_INVALID_ARGUMENT;
+    if (scale) *scale = h->scale;
+    if (good) *good = h->good;
+    if (t) *t = h->t;
+    return NEOX_OK;
+}
+
+neox_status neox_shard_set_state(neox_shard* h, float scale, int32_t good, int64_t t) {
+    if (!h) return NEOX_ERR_INVALID_ARGUMENT;
+    if (!(scale > 0.0f) || !finite(scale) || good < 0 || t < 0)
+        return fail(h, NEOX_ERR_INVALID_ARGUMENT, "state needs a finite scale > 0, good >= 0, t >= 0");
+    DeviceGuard g(h->device);
+    DevScalars s{};
+    s.scale = scale;
+    s.scale_used = scale;
+    s.good = good;
+    s.t = t;
+    cudaError_t e = cudaMemcpy(h->d_sc, &s, sizeof(s), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(h, e, "cudaMemcpy scalars");
+    h->scale = scale;
+    h->good = good;
+    h->t = t;
+    return NEOX_OK;
+}
+
+neox_status neox_shard_set_profiling(neox_shard* h, int32_t enable) {
+    if (!h) return NEOX_ERR_INVALID_ARGUMENT;
+    h->profiling = enable != 0;
+    return NEOX_OK;
+}
+
+neox_status neox_shard_get_profile(const neox_shard* h, neox_profile* out) {
+    if (!h || !out) return NEOX_ERR_INVALID_ARGUMENT;
+    *out = h->prof;
+    return NEOX_OK;
+}
+
+neox_status neox_shard_reset_profile(neox_shard* h) {
+    if (!h) return NEOX_ERR_INVALID_ARGUMENT;
+    const int64_t launches = h->prof.launches;
+    h->prof = neox_profile{};
+    h->prof.launches = launches;
+    return NEOX_OK;
+}
+
+neox_status neox_shard_step(neox_shard* h, const void* const* grads, int32_t num_grads, void* params, float lr,
+                            void* cuda_stream, neox_step_result* out) {
+    if (!h) return NEOX_ERR_INVALID_ARGUMENT;
+    h->last_error.clear();
+    if (!out) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "out is NULL");
+    if (num_grads < 1 || num_grads > kMaxGrads) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "num_grads must be in [1, 64]");
+    if (!grads) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "grads is NULL");
+    if (!finite(lr) || lr < 0.0f) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "lr must be finite and >= 0");
+    GradPtrs gp{};
+    uintptr_t a16[kMaxGrads + 1];
+    if (h->numel > 0) {
+        if (!params) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "params is NULL");
+        if ((uintptr_t)params & 1u) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "params must be 2-byte aligned");
+        for (int k = 0; k < num_grads; k++) {
+            if (!grads[k]) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "grads[" + std::to_string(k) + "] is NULL");
+            if ((uintptr_t)grads[k] & 1u)
+                return fail(h, NEOX_ERR_INVALID_ARGUMENT, "grads[" + std::to_string(k) + "] must be 2-byte aligned");
+            gp.p[k] = static_cast<const uint16_t*>(grads[k]);
+            a16[k] = (uintptr_t)grads[k];
+        }
+        a16[num_grads] = (uintptr_t)params;
+    }
+    DeviceGuard g(h->device);
+    if (!g.ok) return fail(h, NEOX_ERR_CUDA, "cudaSetDevice failed");
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+
+    const bool use_acc = num_grads >= 5 && h->d_acc != nullptr;
+    uintptr_t a32[3] = {(uintptr_t)h->master, (uintptr_t)h->m, (uintptr_t)h->v};
+    int vec = 1;
+    Layout L = h->numel > 0 ? choose_layout(h->numel, a16, num_grads + 1, a32, 3, vec) : Layout{0, 0, 0, 0};
+    float* acc = nullptr;
+    if (use_acc) {
+        const unsigned long long hh = L.head % 4;
+        acc = h->d_acc + ((4 - hh) % 4);  // &acc[head] is 16-byte aligned
+    }
+
+    ScalerArgs sa;
+    sa.post = (double)num_grads / (double)h->hp.predivide;
+    sa.inv_pre = (float)(1.0 / (double)h->hp.predivide);
+    sa.clip = h->hp.clip_norm;
+    sa.factor = h->hp.scale_factor;
+    sa.min_scale = h->hp.min_scale;
+    sa.window = h->hp.scale_window;
+
+    AdamArgs a;
+    a.lr = lr;
+    a.b1 = h->hp.beta1;
+    a.b2 = h->hp.beta2;
+    a.omb1 = 1.0f - h->hp.beta1;
+    a.omb2 = 1.0f - h->hp.beta2;
+    a.eps = h->hp.eps;
+    {
+        const double t1 = (double)(h->t + 1);  // the step count if this step is applied
+        const double bc1 = 1.0 - std::pow((double)h->hp.beta1, t1);
+        const double bc2 = 1.0 - std::pow((double)h->hp.beta2, t1);
+        a.step_size = (float)((double)lr / bc1);
+        a.bcs = (float)std::sqrt(bc2);
+    }
+    a.inv_pre = sa.inv_pre;
+    a.post = sa.post;
+
+    cudaError_t e;
+    if (h->profiling && (e = cudaEventRecord(h->ev[0], st)) != cudaSuccess) return cuda_fail(h, e, "cudaEventRecord");
+    if (h->gdtype == NEOX_FP16) e = dispatch1v<F16>(h, vec, gp, num_grads, L, sa, acc, st);
+    else e = dispatch1v<BF16>(h, vec, gp, num_grads, L, sa, acc, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "pass-1 launch");
+    h->prof.launches += 1;
+    if (h->profiling && (e = cudaEventRecord(h->ev[1], st)) != cudaSuccess) return cuda_fail(h, e, "cudaEventRecord");
+    if (h->numel > 0) {
+        uint16_t* w = static_cast<uint16_t*>(params);
+        if (h->gdtype == NEOX_FP16) {
+            e = h->wdtype == NEOX_FP16 ? dispatch2v<F16, F16>(h, vec, gp, num_grads, acc, L, a, w, st)
+                                       : dispatch2v<F16, BF16>(h, vec, gp, num_grads, acc, L, a, w, st);
+        } else {
+            e = h->wdtype == NEOX_FP16 ? dispatch2v<BF16, F16>(h, vec, gp, num_grads, acc, L, a, w, st)
+                                       : dispatch2v<BF16, BF16>(h, vec, gp, num_grads, acc, L, a, w, st);
+        }
+        if (e != cudaSuccess) return cuda_fail(h, e, "pass-2 launch");
+        h->prof.launches += 1;
+    }
+    if (h->profiling && (e = cudaEventRecord(h->ev[2], st)) != cudaSuccess) return cuda_fail(h, e, "cudaEventRecord");
+    if ((e = cudaMemcpyAsync(h->h_sc, h->d_sc, sizeof(DevScalars), cudaMemcpyDeviceToHost, st)) != cudaSuccess)
+        return cuda_fail(h, e, "cudaMemcpyAsync result");
+    if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(h, e, "step execution");
+
+    const DevScalars& r = *h->h_sc;
+    out->overflow = r.overflow;
+    out->grad_norm = r.norm;
+    out->clip_coef = r.coef;
+    out->loss_scale = r.scale_used;
+    out->loss_scale_next = r.scale;
+    out->good_steps = r.good;
+    out->applied_steps = r.t;
+    h->scale = r.scale;
+    h->good = r.good;
+    h->t = r.t;
+
+    if (h->profiling) {
+        float t01 = 0.f, t12 = 0.f;
+        cudaEventElapsedTime(&t01, h->ev[0], h->ev[1]);
+        cudaEventElapsedTime(&t12, h->ev[1], h->ev[2]);
+        h->prof.steps += 1;
+        h->prof.grad_pass_ms += t01;
+        h->prof.update_pass_ms += t12;
+        h->prof.last_grad_pass_ms = t01;
+        h->prof.last_update_pass_ms = t12;
+    }
+    return NEOX_OK;
+}
+
+}  // extern "C"

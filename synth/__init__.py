@@ -138,3 +138,87 @@ def rate_inject_mask(n: int, rate: float, seed: int, tensor_id: int, step: int, 
     hit = x[0] < thresh
     kind = (x[1] % np.uint32(3)).astype(np.int64)
     return hit, kind
+
+
+# ---------------------------------------------------------------------------
+# GPU generator (synth/philox_gen.cu), for inputs at full size.  Outputs are
+# written into caller-provided torch CUDA tensors on torch's current stream.
+# ---------------------------------------------------------------------------
+import ctypes as _ct
+import os as _os
+import subprocess as _sp
+
+_HERE = _os.path.dirname(_os.path.abspath(__file__))
+_CU = _os.path.join(_HERE, "philox_gen.cu")
+_SO = _os.path.join(_HERE, "libsynth.so")
+_gpu_lib = None
+
+
+def build_cuda(force: bool = False) -> str:
+    if force or not _os.path.exists(_SO) or _os.path.getmtime(_SO) < _os.path.getmtime(_CU):
+        tmp = _SO + f".tmp{_os.getpid()}"
+        _sp.check_call(["/usr/local/cuda/bin/nvcc", "-gencode", "arch=compute_100a,code=sm_100a", "-O3",
+                        "-lineinfo", "-Xcompiler", "-fPIC", "-shared", "-o", tmp, _CU])
+        _os.replace(tmp, _SO)
+    return _SO
+
+
+def _lib():
+    global _gpu_lib
+    if _gpu_lib is None:
+        if not _os.path.exists(_SO):
+            build_cuda()
+        L = _ct.CDLL(_SO)
+        u64, u32, f, i, p = _ct.c_ulonglong, _ct.c_uint32, _ct.c_float, _ct.c_int, _ct.c_void_p
+        L.synth_normal16.argtypes = [p, u64, u64, f, f, u32, u32, u32, i, p]
+        L.synth_normal32.argtypes = [p, u64, u64, f, u32, u32, u32, p]
+        L.synth_t3_16.argtypes = [p, u64, u64, f, u32, u32, u32, i, p]
+        L.synth_rate_inject16.argtypes = [p, u64, u64, u32, u32, u32, u32, i, p, p]
+        L.synth_philox_raw.argtypes = [p, u64, u32, u32, u32, p]
+        _gpu_lib = L
+    return _gpu_lib
+
+
+def _stream():
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise RuntimeError(f"{what}: CUDA error {rc}")
+
+
+def gpu_grad_normal16(out, sigma, scale, seed, tensor_id, step, bf16=False, start=0):
+    """out (16-bit CUDA tensor) <- RNE16(fl32(z*sigma)*scale), z the Philox normals."""
+    _check(_lib().synth_normal16(out.data_ptr(), out.numel(), start, sigma, scale, seed,
+                                 STREAM_GRAD | (tensor_id << 8), step, int(bf16), _stream()), "synth_normal16")
+
+
+def gpu_grad_t3_16(out, scale, seed, tensor_id, step, bf16=False, start=0):
+    _check(_lib().synth_t3_16(out.data_ptr(), out.numel(), start, scale, seed,
+                              STREAM_GRAD | (tensor_id << 8), step, int(bf16), _stream()), "synth_t3_16")
+
+
+def gpu_master_normal(out, sigma, seed, tensor_id=0, start=0):
+    _check(_lib().synth_normal32(out.data_ptr(), out.numel(), start, sigma, seed,
+                                 STREAM_MASTER | (tensor_id << 8), 0, _stream()), "synth_normal32")
+
+
+def gpu_rate_inject(out, rate, seed, tensor_id, step, bf16=False, start=0) -> int:
+    """Overwrite each element with +inf / NaN / -inf with probability `rate`; returns the hit count."""
+    import torch
+    hits = torch.zeros(1, dtype=torch.int64, device=out.device)
+    thresh = min(int(rate * 2.0 ** 32), 0xFFFFFFFF)
+    _check(_lib().synth_rate_inject16(out.data_ptr(), out.numel(), start, thresh, seed,
+                                      STREAM_INJECT_RATE | (tensor_id << 8), step, int(bf16),
+                                      hits.data_ptr(), _stream()), "synth_rate_inject16")
+    return int(hits.item())
+
+
+def gpu_philox_raw(nblocks: int, step: int, seed: int, stream: int):
+    """Raw Philox output of counters (b, step) for b < nblocks, as uint32 numpy [nblocks, 4]."""
+    import torch
+    out = torch.empty(nblocks * 4, dtype=torch.int32, device="cuda")
+    _check(_lib().synth_philox_raw(out.data_ptr(), nblocks, step, seed, stream, _stream()), "synth_philox_raw")
+    return out.cpu().numpy().view(np.uint32).reshape(nblocks, 4)

@@ -1,0 +1,119 @@
+"""Host-side checks of the C ABI library that need no GPU: it loads, it exports
+every function include/neox_shard.h declares, its host arithmetic and its
+argument validation (which runs before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mixed_precision_zero_b200 import _abi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+GOLDEN = os.path.join(ROOT, "tests", "golden")
+
+
+def declared_functions():
+    names = []
+    inc = os.path.join(ROOT, "include")
+    for fn in sorted(os.listdir(inc)):
+        if not fn.endswith(".h"):
+            continue
+        text = open(os.path.join(inc, fn)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(neox_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_function():
+    names = declared_functions()
+    assert "neox_shard_step" in names and "neox_shard_create" in names and len(names) >= 10
+    L = ctypes.CDLL(_abi.LIB_PATH)
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_state_accounting_matches_page():
+    """16 bytes per parameter: 175B parameters -> 2.8 TB, FP16 weights 350 GB."""
+    facts = dict(ln.split() for ln in open(os.path.join(GOLDEN, "state_accounting.txt"))
+                 if ln.strip() and not ln.startswith("#"))
+    n = int(facts["params"])
+    assert _abi.neox_model_state_bytes(n, _abi.NEOX_FP16, _abi.NEOX_FP16) == int(facts["state_bytes"])
+    assert _abi.neox_model_state_bytes(n, _abi.NEOX_BF16, _abi.NEOX_BF16) == int(facts["state_bytes"])
+    assert 2 * n == int(facts["fp16_weight_bytes"])
+
+
+def test_status_strings():
+    for s in range(5):
+        assert _abi.neox_status_string(s)
+    assert _abi.neox_status_string(99) == "unknown status"
+
+
+def _desc(n=16, **kw):
+    d = _abi.neox_shard_desc()
+    d.numel = n
+    d.wdtype = kw.get("wdtype", _abi.NEOX_FP16)
+    d.gdtype = kw.get("gdtype", _abi.NEOX_FP16)
+    d.master = kw.get("master", 4096)
+    d.exp_avg = kw.get("exp_avg", 8192)
+    d.exp_avg_sq = kw.get("exp_avg_sq", 12288)
+    d.default_weight_decay = kw.get("wd", 0.1)
+    d.max_grads = kw.get("max_grads", 1)
+    return d
+
+
+def _hp(**kw):
+    base = dict(beta1=0.9, beta2=0.95, eps=1e-8, clip_norm=1.0, predivide=1.0, init_scale=65536.0,
+                scale_factor=2.0, min_scale=1.0, scale_window=1000)
+    base.update(kw)
+    return _abi.neox_hparams(**base)
+
+
+@pytest.mark.parametrize("desc_kw,hp_kw,why", [
+    ({}, {"beta1": 1.0}, "beta1"),
+    ({}, {"beta2": -0.1}, "beta2"),
+    ({}, {"eps": float("nan")}, "eps"),
+    ({}, {"predivide": 0.0}, "predivide"),
+    ({}, {"init_scale": 0.0}, "init_scale"),
+    ({}, {"scale_factor": 0.5}, "scale_factor"),
+    ({}, {"min_scale": -1.0}, "min_scale"),
+    ({}, {"scale_window": 0}, "scale_window"),
+    ({"wdtype": 7}, {}, "dtype"),
+    ({"master": 0}, {}, "non-NULL"),
+    ({"exp_avg": 8194}, {}, "aligned"),
+    ({"max_grads": 65}, {}, "max_grads"),
+    ({"wd": float("inf")}, {}, "weight decay"),
+])
+def test_create_rejects_invalid_arguments_before_cuda(desc_kw, hp_kw, why):
+    h = ctypes.c_void_p()
+    st = _abi.lib().neox_shard_create(ctypes.byref(_desc(**desc_kw)), ctypes.byref(_hp(**hp_kw)), 0,
+                                      ctypes.byref(h))
+    assert st == _abi.NEOX_ERR_INVALID_ARGUMENT
+    assert h.value is None
+    assert why in _abi.neox_last_error(None)
+
+
+def test_create_rejects_bad_segment_tables():
+    L = _abi.lib()
+    for segs in ([(0, 8, 0.1), (9, 8, 0.1)], [(0, 8, 0.1), (8, 0, 0.1), (8, 8, 0.1)], [(0, 15, 0.1)],
+                 [(1, 16, 0.1)]):
+        arr = (_abi.neox_segment * len(segs))(*[_abi.neox_segment(*s) for s in segs])
+        d = _desc(16)
+        d.segs = ctypes.cast(arr, ctypes.POINTER(_abi.neox_segment))
+        d.nsegs = len(segs)
+        h = ctypes.c_void_p()
+        assert L.neox_shard_create(ctypes.byref(d), ctypes.byref(_hp()), 0, ctypes.byref(h)) == \
+            _abi.NEOX_ERR_INVALID_ARGUMENT
+    for bad in (None,):
+        assert L.neox_shard_create(None, ctypes.byref(_hp()), 0, ctypes.byref(ctypes.c_void_p())) == \
+            _abi.NEOX_ERR_INVALID_ARGUMENT
+
+
+def test_null_handle_calls():
+    L = _abi.lib()
+    assert L.neox_shard_step(None, None, 1, None, 1e-3, None, None) == _abi.NEOX_ERR_INVALID_ARGUMENT
+    assert L.neox_shard_set_state(None, 1.0, 0, 0) == _abi.NEOX_ERR_INVALID_ARGUMENT
+    assert L.neox_shard_get_state(None, None, None, None) == _abi.NEOX_ERR_INVALID_ARGUMENT
+    assert L.neox_shard_set_hparams(None, None) == _abi.NEOX_ERR_INVALID_ARGUMENT
+    assert L.neox_shard_scratch_bytes(None) == 0
+    L.neox_shard_destroy(None)
