@@ -184,6 +184,59 @@ neox_status neox_shard_set_profiling(neox_shard* h, int32_t enable);
 neox_status neox_shard_get_profile(const neox_shard* h, neox_profile* out);
 neox_status neox_shard_reset_profile(neox_shard* h);
 
+/* ------------------------------------------------------------------------
+ * Step without a handle and without any allocation.
+ *
+ * The pages have no counterpart to this entry point; it is a library service.
+ * Some callers may not allocate device or pinned memory at all: code running
+ * inside a device-memory allocator's own hook (a cudaMalloc there re-enters
+ * the allocator), runtimes that give all device memory to their own pool up
+ * front, and loops that must not let cudaMalloc / cudaFree synchronise the
+ * device.  neox_shard_create allocates, so those callers use this function
+ * instead.  It runs the same two kernels as neox_shard_step and calls no
+ * cudaMalloc, cudaMallocHost, cudaFree or other allocating routine.  Its
+ * scratch (per-block partial sums, the 64-byte scalar block, the segment
+ * table) is one static device array of about 68 KiB, which every GPU that
+ * loads this library holds until the process exits.
+ *
+ * Limits: at most 1024 segments (a longer table is rejected with
+ * NEOX_ERR_INVALID_ARGUMENT and a message); K in [1, 64].  There is no FP32
+ * gradient-sum buffer (it would need numel*4 bytes), so K >= 5 re-reads the K
+ * buffers in pass 2; desc->max_grads is ignored.  numel itself is not limited.
+ *
+ * Arguments are those of neox_shard_create + neox_shard_step; desc->numel,
+ * dtypes, segment table and the caller-owned master / exp_avg / exp_avg_sq
+ * describe the shard.  *state carries the loss-scaler state in (the scale this
+ * step's gradients carry, the counter, t) and receives it back after the step;
+ * start with {init_scale, 0, 0}.  hp->init_scale is ignored.  Runs on the
+ * calling thread's current CUDA device and on cuda_stream; returns after the
+ * step has finished (it synchronises cuda_stream only).
+ *
+ * Set-up: the first call on each device looks up the address of the static
+ * array on that device (cudaGetSymbolAddress); make that first call before any
+ * stream capture begins.
+ *
+ * Sharing: every call on a device uses the same static array, and the array
+ * keeps the previous call's contents.  Each call reloads what must start
+ * fresh (the scalar block with its ticket counter set to zero, and the segment
+ * table) on its own stream, so calls one after another are independent.  Calls
+ * that overlap on the GPU (concurrent streams, or threads calling at the same
+ * time) race on the array and give wrong results: serialise them.
+ *
+ * Errors as neox_shard_step; the message of the last failed call on this
+ * thread is neox_noalloc_last_error().
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    float scale;     /* loss scale the step's gradients carry (> 0)   */
+    int32_t good;    /* consecutive applied steps (>= 0)               */
+    int64_t t;       /* applied steps so far (>= 0)                    */
+} neox_scaler_state;
+
+neox_status neox_shard_step_noalloc(const neox_shard_desc* desc, const neox_hparams* hp,
+                                    neox_scaler_state* state, const void* const* grads, int32_t num_grads,
+                                    void* params, float lr, void* cuda_stream, neox_step_result* out);
+const char* neox_noalloc_last_error(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -49,6 +49,10 @@ class neox_step_result(ctypes.Structure):
         return {k: getattr(self, k) for k, _ in self._fields_}
 
 
+class neox_scaler_state(ctypes.Structure):
+    _fields_ = [("scale", ctypes.c_float), ("good", ctypes.c_int32), ("t", ctypes.c_int64)]
+
+
 class neox_profile(ctypes.Structure):
     _fields_ = [("steps", ctypes.c_int64), ("launches", ctypes.c_int64),
                 ("grad_pass_ms", ctypes.c_double), ("update_pass_ms", ctypes.c_double),
@@ -97,6 +101,13 @@ def lib() -> ctypes.CDLL:
         L.neox_shard_get_profile.restype = S
         L.neox_shard_reset_profile.argtypes = [_H]
         L.neox_shard_reset_profile.restype = S
+        L.neox_shard_step_noalloc.argtypes = [ctypes.POINTER(neox_shard_desc), ctypes.POINTER(neox_hparams),
+                                              ctypes.POINTER(neox_scaler_state), ctypes.POINTER(ctypes.c_void_p),
+                                              ctypes.c_int32, ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p,
+                                              ctypes.POINTER(neox_step_result)]
+        L.neox_shard_step_noalloc.restype = S
+        L.neox_noalloc_last_error.argtypes = []
+        L.neox_noalloc_last_error.restype = ctypes.c_char_p
         _lib = L
     return _lib
 
@@ -178,3 +189,15 @@ def neox_shard_get_profile(h: int) -> neox_profile:
 
 def neox_shard_reset_profile(h: int) -> None:
     lib().neox_shard_reset_profile(h)
+
+
+def neox_shard_step_noalloc(desc: neox_shard_desc, hp: neox_hparams, state: neox_scaler_state, grad_ptrs,
+                            params_ptr: int, lr: float, stream: int) -> neox_step_result:
+    """The step without a handle or any allocation; `state` is updated in place."""
+    arr = (ctypes.c_void_p * len(grad_ptrs))(*grad_ptrs)
+    res = neox_step_result()
+    st = lib().neox_shard_step_noalloc(ctypes.byref(desc), ctypes.byref(hp), ctypes.byref(state), arr,
+                                       len(grad_ptrs), params_ptr, lr, stream, ctypes.byref(res))
+    if st != NEOX_OK:
+        raise NeoxError(st, lib().neox_noalloc_last_error().decode())
+    return res

@@ -949,3 +949,235 @@ neox_status neox_shard_step(neox_shard* h, const void* const* grads, int32_t num
 }
 
 }  // extern "C"
+
+// ====================================================================== no-allocation step
+//
+// neox_shard_step_noalloc runs the same two kernels as neox_shard_step, but
+// without a handle and without allocating anything: the per-block partial
+// sums, the scalar block and the segment table live in one file-scope static
+// device array instead of memory obtained from cudaMalloc at create time.  It
+// exists for callers that must not allocate device or pinned memory, e.g. code
+// running inside an allocator's own hook (a cudaMalloc there would re-enter
+// the allocator), runtimes that hand the whole device memory to their own pool
+// up front, and latency-critical loops where cudaMalloc / cudaFree would
+// synchronise the device.
+
+#include <mutex>
+
+namespace {
+
+constexpr int kNoallocMaxSegments = 1024;
+constexpr int kNoallocMaxParts = 148 * kMaxBlocksPerSm;  // one slot per pass-1 block on a B200
+constexpr int kNoallocMaxDevices = 64;
+
+// Byte layout of the static scratch.
+constexpr size_t kNaOffScalars = 0;
+constexpr size_t kNaOffPartS = 256;
+constexpr size_t kNaOffPartB = kNaOffPartS + sizeof(double) * kNoallocMaxParts;
+constexpr size_t kNaOffSegEnd = (kNaOffPartB + sizeof(int) * kNoallocMaxParts + 255) / 256 * 256;
+constexpr size_t kNaOffSegWd = kNaOffSegEnd + sizeof(unsigned long long) * kNoallocMaxSegments;
+constexpr size_t kNoallocScratchBytes = (kNaOffSegWd + sizeof(float) * kNoallocMaxSegments + 255) / 256 * 256;
+
+// Every GPU that loads this library holds these bytes (about 68 KiB) until the process exits.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+struct NoallocDevice {
+    bool ready = false;
+    unsigned char* base = nullptr;  // device address of g_noalloc_scratch on this device
+    int sm_count = 0;
+};
+NoallocDevice g_noalloc_dev[kNoallocMaxDevices];
+std::mutex g_noalloc_mu;
+thread_local char g_noalloc_error[256];
+
+neox_status noalloc_fail(neox_status st, const char* fmt, long long a = 0, long long b = 0) {
+    snprintf(g_noalloc_error, sizeof(g_noalloc_error), fmt, a, b);
+    return st;
+}
+
+// Once per device, with that device current: look up where the static scratch
+// lives on it (host code cannot use the array's name as a device address).
+neox_status noalloc_setup(int dev, NoallocDevice** out) {
+    if (dev < 0 || dev >= kNoallocMaxDevices) return noalloc_fail(NEOX_ERR_UNSUPPORTED, "device index beyond 63");
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    NoallocDevice& d = g_noalloc_dev[dev];
+    if (!d.ready) {
+        int major = 0, sms = 0;
+        cudaError_t e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess)
+            return noalloc_fail(NEOX_ERR_CUDA, "cudaDeviceGetAttribute failed (cudaError %lld)", (long long)e);
+        if (major != 10) return noalloc_fail(NEOX_ERR_UNSUPPORTED, "this library is built for sm_100a (B200)");
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || p == nullptr)
+            return noalloc_fail(NEOX_ERR_CUDA, "cudaGetSymbolAddress failed (cudaError %lld)", (long long)e);
+        d.base = static_cast<unsigned char*>(p);
+        d.sm_count = sms;
+        d.ready = true;
+    }
+    *out = &d;
+    return NEOX_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* neox_noalloc_last_error(void) { return g_noalloc_error; }
+
+neox_status neox_shard_step_noalloc(const neox_shard_desc* d, const neox_hparams* hp, neox_scaler_state* state,
+                                    const void* const* grads, int32_t num_grads, void* params, float lr,
+                                    void* cuda_stream, neox_step_result* out) {
+    g_noalloc_error[0] = 0;
+    if (!d || !state || !out) return noalloc_fail(NEOX_ERR_INVALID_ARGUMENT, "desc, state and out must be non-NULL");
+    if (const char* why = check_hparams(hp)) {
+        snprintf(g_noalloc_error, sizeof(g_noalloc_error), "%s", why);
+        return NEOX_ERR_INVALID_ARGUMENT;
+    }
+    if ((d->wdtype != NEOX_FP16 && d->wdtype != NEOX_BF16) || (d->gdtype != NEOX_FP16 && d->gdtype != NEOX_BF16))
+        return noalloc_fail(NEOX_ERR_INVALID_ARGUMENT, "dtype must be NEOX_FP16 or NEOX_BF16");
+    if (!(state->scale > 0.0f) || !finite(state->scale) || state->good < 0 || state->t < 0)
+        return noalloc_fail(NEOX_ERR_INVALID_ARGUMENT, "state needs a finite scale > 0, good >= 0, t >= 0");
+    if (num_grads < 1 || num_grads > kMaxGrads) return noalloc_fail(NEOX_ERR_INVALID_ARGUMENT, "num_grads must be in [1, 64]");
+    if (!grads) return noalloc_fail(NEOX_ERR_INVALID_ARGUMENT, "grads is NULL");
+    if (!finite(lr) || lr < 0.0f) return noalloc_fail(NEOX_ERR_INVALID_ARGUMENT, "lr must be finite and >= 0");
+    if (!finite(d->default_weight_decay)) return noalloc_fail(NEOX_ERR_INVALID_ARGUMENT, "weight decay must be finite");
+    const int nsegs = d->segs ? d->nsegs : 1;
+    if (d->segs && nsegs < 1) return noalloc_fail(NEOX_ERR_INVALID_ARGUMENT, "nsegs must be >= 1 with a table");
+    if (nsegs > kNoallocMaxSegments)
+        return noalloc_fail(NEOX_ERR_INVALID_ARGUMENT,
+                            "segment table of %lld entries exceeds the static scratch maximum of %lld segments",
+                            nsegs, kNoallocMaxSegments);
+    unsigned long long ends[kNoallocMaxSegments];
+    float wds[kNoallocMaxSegments];
+    if (d->segs) {
+        unsigned long long pos = 0;
+        for (int i = 0; i < nsegs; i++) {
+            const neox_segment& s = d->segs[i];
+            if (s.offset != pos || s.numel == 0 || !finite(s.weight_decay))
+                return noalloc_fail(NEOX_ERR_INVALID_ARGUMENT, "segments must be sorted, non-empty, finite and tile [0, numel)");
+            pos += s.numel;
+            ends[i] = pos;
+            wds[i] = s.weight_decay;
+        }
+        if (pos != d->numel) return noalloc_fail(NEOX_ERR_INVALID_ARGUMENT, "segments do not cover numel");
+    } else {
+        ends[0] = d->numel;
+        wds[0] = d->default_weight_decay;
+    }
+    GradPtrs gp{};
+    uintptr_t a16[kMaxGrads + 1];
+    if (d->numel > 0) {
+        if (!d->master || !d->exp_avg || !d->exp_avg_sq || !params)
+            return noalloc_fail(NEOX_ERR_INVALID_ARGUMENT, "master/exp_avg/exp_avg_sq/params must be non-NULL");
+        if (((uintptr_t)d->master | (uintptr_t)d->exp_avg | (uintptr_t)d->exp_avg_sq) & 3u)
+            return noalloc_fail(NEOX_ERR_INVALID_ARGUMENT, "FP32 state arrays must be 4-byte aligned");
+        if ((uintptr_t)params & 1u) return noalloc_fail(NEOX_ERR_INVALID_ARGUMENT, "params must be 2-byte aligned");
+        for (int k = 0; k < num_grads; k++) {
+            if (!grads[k] || ((uintptr_t)grads[k] & 1u))
+                return noalloc_fail(NEOX_ERR_INVALID_ARGUMENT, "grads[%lld] is NULL or not 2-byte aligned", k);
+            gp.p[k] = static_cast<const uint16_t*>(grads[k]);
+            a16[k] = (uintptr_t)grads[k];
+        }
+        a16[num_grads] = (uintptr_t)params;
+    }
+
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return noalloc_fail(NEOX_ERR_CUDA, "cudaGetDevice failed (cudaError %lld)", (long long)e);
+    NoallocDevice* nd = nullptr;
+    if (neox_status s = noalloc_setup(dev, &nd); s != NEOX_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+
+    // A view of the static scratch shaped like a handle, so the launches below
+    // are exactly those of neox_shard_step.  Nothing here allocates.
+    neox_shard v;
+    v.device = dev;
+    v.sm_count = nd->sm_count;
+    v.max_parts = nd->sm_count * kMaxBlocksPerSm < kNoallocMaxParts ? nd->sm_count * kMaxBlocksPerSm : kNoallocMaxParts;
+    v.numel = d->numel;
+    v.master = d->master;
+    v.m = d->exp_avg;
+    v.v = d->exp_avg_sq;
+    v.d_sc = reinterpret_cast<DevScalars*>(nd->base + kNaOffScalars);
+    v.d_part_s = reinterpret_cast<double*>(nd->base + kNaOffPartS);
+    v.d_part_b = reinterpret_cast<int*>(nd->base + kNaOffPartB);
+    v.d_seg_end = reinterpret_cast<unsigned long long*>(nd->base + kNaOffSegEnd);
+    v.d_seg_wd = reinterpret_cast<float*>(nd->base + kNaOffSegWd);
+    v.nsegs = nsegs;
+
+    // The scratch keeps the previous call's contents: reload the scaler block
+    // (ticket counter back to zero) and the segment table on this stream.
+    DevScalars init{};
+    init.scale = state->scale;
+    init.scale_used = state->scale;
+    init.good = state->good;
+    init.t = state->t;
+    if ((e = cudaMemcpyAsync(v.d_sc, &init, sizeof(init), cudaMemcpyHostToDevice, st)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(v.d_seg_end, ends, sizeof(unsigned long long) * nsegs, cudaMemcpyHostToDevice, st)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(v.d_seg_wd, wds, sizeof(float) * nsegs, cudaMemcpyHostToDevice, st)) != cudaSuccess)
+        return noalloc_fail(NEOX_ERR_CUDA, "staging the scratch failed (cudaError %lld)", (long long)e);
+
+    uintptr_t a32[3] = {(uintptr_t)d->master, (uintptr_t)d->exp_avg, (uintptr_t)d->exp_avg_sq};
+    int vec = 1;
+    Layout L = d->numel > 0 ? choose_layout(d->numel, a16, num_grads + 1, a32, 3, vec) : Layout{0, 0, 0, 0};
+
+    ScalerArgs sa;
+    sa.post = (double)num_grads / (double)hp->predivide;
+    sa.inv_pre = (float)(1.0 / (double)hp->predivide);
+    sa.clip = hp->clip_norm;
+    sa.factor = hp->scale_factor;
+    sa.min_scale = hp->min_scale;
+    sa.window = hp->scale_window;
+    AdamArgs a;
+    a.lr = lr;
+    a.b1 = hp->beta1;
+    a.b2 = hp->beta2;
+    a.omb1 = 1.0f - hp->beta1;
+    a.omb2 = 1.0f - hp->beta2;
+    a.eps = hp->eps;
+    {
+        const double t1 = (double)(state->t + 1);
+        const double bc1 = 1.0 - std::pow((double)hp->beta1, t1);
+        const double bc2 = 1.0 - std::pow((double)hp->beta2, t1);
+        a.step_size = (float)((double)lr / bc1);
+        a.bcs = (float)std::sqrt(bc2);
+    }
+    a.inv_pre = sa.inv_pre;
+    a.post = sa.post;
+
+    // K >= 5 re-reads the K buffers in pass 2 (no FP32-sum buffer: it would
+    // need numel * 4 bytes of scratch).
+    e = d->gdtype == NEOX_FP16 ? dispatch1v<F16>(&v, vec, gp, num_grads, L, sa, nullptr, st)
+                               : dispatch1v<BF16>(&v, vec, gp, num_grads, L, sa, nullptr, st);
+    if (e != cudaSuccess) return noalloc_fail(NEOX_ERR_CUDA, "pass-1 launch failed (cudaError %lld)", (long long)e);
+    if (d->numel > 0) {
+        uint16_t* w = static_cast<uint16_t*>(params);
+        if (d->gdtype == NEOX_FP16) {
+            e = d->wdtype == NEOX_FP16 ? dispatch2v<F16, F16>(&v, vec, gp, num_grads, nullptr, L, a, w, st)
+                                       : dispatch2v<F16, BF16>(&v, vec, gp, num_grads, nullptr, L, a, w, st);
+        } else {
+            e = d->wdtype == NEOX_FP16 ? dispatch2v<BF16, F16>(&v, vec, gp, num_grads, nullptr, L, a, w, st)
+                                       : dispatch2v<BF16, BF16>(&v, vec, gp, num_grads, nullptr, L, a, w, st);
+        }
+        if (e != cudaSuccess) return noalloc_fail(NEOX_ERR_CUDA, "pass-2 launch failed (cudaError %lld)", (long long)e);
+    }
+    DevScalars r{};
+    if ((e = cudaMemcpyAsync(&r, v.d_sc, sizeof(r), cudaMemcpyDeviceToHost, st)) != cudaSuccess ||
+        (e = cudaStreamSynchronize(st)) != cudaSuccess)
+        return noalloc_fail(NEOX_ERR_CUDA, "step execution failed (cudaError %lld)", (long long)e);
+    out->overflow = r.overflow;
+    out->grad_norm = r.norm;
+    out->clip_coef = r.coef;
+    out->loss_scale = r.scale_used;
+    out->loss_scale_next = r.scale;
+    out->good_steps = r.good;
+    out->applied_steps = r.t;
+    state->scale = r.scale;
+    state->good = r.good;
+    state->t = r.t;
+    return NEOX_OK;
+}
+
+}  // extern "C"
