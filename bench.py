@@ -394,7 +394,8 @@ def run_b200(args):
         "dtype": "f32", "data": "synthetic",
         "config": {"workload": wl.name, "numel_per_rank": wl.numel, "segments": len(wl.segments or [1]),
                    "grad_buffers": wl.K, "weights": "bf16" if wl.bf16 else "fp16",
-                   "state": "fp32 master/m/v", "l2": "inputs 22.6 GB per rank >> 126 MB L2; no flush",
+                   "state": "fp32 master/m/v",
+                   "l2": f"inputs {(14 + 2 * wl.K) * wl.numel / 1e9:.1f} GB per rank >> 126 MB L2; no flush",
                    "parallelism": f"{ws} independent shard(s), one per GPU"},
         "hbm": {"step_gbs": step_gbs, "step_frac": step_gbs / peak, "bytes_per_param": p1b + p2b,
                 "peak_gbs": peak, "peak_kind": peak_kind},

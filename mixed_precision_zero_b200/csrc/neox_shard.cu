@@ -47,7 +47,9 @@ namespace {
 
 constexpr int kMaxGrads = 64;
 constexpr int kThreads1 = 512;   // pass-1 block
+constexpr int kUnroll1 = 4;      // pass-1 vectors in flight per thread
 constexpr int kThreads3 = 256;   // pass-2 block
+constexpr int kUnroll3 = 1;      // pass-2 vectors in flight per thread
 constexpr int kMaxBlocksPerSm = 32;
 
 struct GradPtrs {
@@ -197,6 +199,32 @@ __device__ __forceinline__ void ingest(const GradPtrs& gp, int K, unsigned long 
     for (int e = 0; e < VEC; e++) g[e] = __fmul_rn(g[e], inv_us);
 }
 
+// U vectors at global indices i0, i0 + di, ..., ingested together: for every
+// buffer the U loads are issued before any of them is used, so each thread
+// keeps U 16-byte requests in flight.  Per element the arithmetic (and its
+// order over buffers) is that of ingest().
+template <class G, int VEC, int U>
+__device__ __forceinline__ void ingest_batch(const GradPtrs& gp, int K, unsigned long long i0, unsigned long long di,
+                                             float inv_pre, float inv_us, float (&g)[U][VEC]) {
+#pragma unroll
+    for (int u = 0; u < U; u++)
+#pragma unroll
+        for (int e = 0; e < VEC; e++) g[u][e] = 0.0f;
+    for (int k = 0; k < K; k++) {
+        uint16_t h[U][VEC];
+#pragma unroll
+        for (int u = 0; u < U; u++) ld16<VEC>(gp.p[k] + i0 + u * di, h[u]);
+#pragma unroll
+        for (int u = 0; u < U; u++)
+#pragma unroll
+            for (int e = 0; e < VEC; e++) g[u][e] = __fadd_rn(g[u][e], __fmul_rn(G::dec(h[u][e]), inv_pre));
+    }
+#pragma unroll
+    for (int u = 0; u < U; u++)
+#pragma unroll
+        for (int e = 0; e < VEC; e++) g[u][e] = __fmul_rn(g[u][e], inv_us);
+}
+
 __device__ __forceinline__ float unscale_factor(double post, float scale) {
     return (float)(1.0 / (post * (double)scale));
 }
@@ -259,8 +287,20 @@ grad_stats_kernel(GradPtrs gp, int K, Layout L, ScalerArgs sa, float* __restrict
     double s = 0.0;
     int bad = 0;
 
+    // Grid-stride over vectors, kUnroll1 strides per iteration (the thread
+    // still visits its vectors in the same order, so its sum is unchanged).
     const unsigned long long stride = (unsigned long long)gridDim.x * kThreads1;
-    for (unsigned long long v = (unsigned long long)blockIdx.x * kThreads1 + threadIdx.x; v < L.nvec; v += stride) {
+    unsigned long long v = (unsigned long long)blockIdx.x * kThreads1 + threadIdx.x;
+    for (; v + (kUnroll1 - 1) * stride < L.nvec; v += kUnroll1 * stride) {
+        float g[kUnroll1][VEC];
+        ingest_batch<G, VEC, kUnroll1>(gp, K, L.head + v * VEC, stride * VEC, sa.inv_pre, inv_us, g);
+#pragma unroll
+        for (int u = 0; u < kUnroll1; u++) {
+            s += vec_sumsq<VEC>(g[u], bad);
+            if constexpr (WRITE_ACC) st32<VEC>(acc + L.head + (v + u * stride) * VEC, g[u]);
+        }
+    }
+    for (; v < L.nvec; v += stride) {
         const unsigned long long i = L.head + v * VEC;
         float g[VEC];
         ingest<G, VEC>(gp, K, i, sa.inv_pre, inv_us, g);
@@ -394,7 +434,49 @@ adam_kernel(GradPtrs gp, int K, const float* __restrict__ acc, Layout L, AdamArg
     SegCursor cur{0, 0ull, 1.0f};
     if (v0 < L.nvec) seg_seek(cur, L.head + v0 * VEC, seg_end, seg_wd, nsegs, a.lr);
 
-    for (unsigned long long vi = v0; vi < L.nvec; vi += stride) {
+    unsigned long long vi = v0;
+    // kUnroll3 strides per iteration: every load of the batch is issued before
+    // the first update, to keep more bytes in flight per thread.
+    if constexpr (kUnroll3 > 1) {
+        for (; vi + (kUnroll3 - 1) * stride < L.nvec; vi += kUnroll3 * stride) {
+            float g[kUnroll3][VEC], p[kUnroll3][VEC], mm[kUnroll3][VEC], vv[kUnroll3][VEC];
+            if constexpr (READ_ACC) {
+#pragma unroll
+                for (int u = 0; u < kUnroll3; u++) ld32<VEC>(acc + L.head + (vi + u * stride) * VEC, g[u]);
+            } else {
+                ingest_batch<G, VEC, kUnroll3>(gp, K, L.head + vi * VEC, stride * VEC, a.inv_pre, inv_us, g);
+            }
+#pragma unroll
+            for (int u = 0; u < kUnroll3; u++) {
+                const unsigned long long i = L.head + (vi + u * stride) * VEC;
+                ld32<VEC>(master + i, p[u]);
+                ld32<VEC>(m + i, mm[u]);
+                ld32<VEC>(v + i, vv[u]);
+            }
+#pragma unroll
+            for (int u = 0; u < kUnroll3; u++) {
+                const unsigned long long i = L.head + (vi + u * stride) * VEC;
+                float keep[VEC];
+                if (i >= cur.end) seg_seek(cur, i, seg_end, seg_wd, nsegs, a.lr);
+                if (i + VEC <= cur.end) {
+#pragma unroll
+                    for (int e = 0; e < VEC; e++) keep[e] = cur.keep;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < VEC; e++) {
+                        if (i + e >= cur.end) seg_seek(cur, i + e, seg_end, seg_wd, nsegs, a.lr);
+                        keep[e] = cur.keep;
+                    }
+                }
+                adam_vec<VEC>(g[u], keep, c, a, p[u], mm[u], vv[u]);
+                st32<VEC>(master + i, p[u]);
+                st32<VEC>(m + i, mm[u]);
+                st32<VEC>(v + i, vv[u]);
+                st16<W, VEC>(w + i, p[u]);
+            }
+        }
+    }
+    for (; vi < L.nvec; vi += stride) {
         const unsigned long long i = L.head + vi * VEC;
         float g[VEC], p[VEC], mm[VEC], vv[VEC], keep[VEC];
         if constexpr (READ_ACC) ld32<VEC>(acc + i, g);

@@ -85,7 +85,7 @@ def pythia_1p4b(layers=24, hidden=2048, vocab=50304) -> Workload:
     """Pythia-1.4B-shaped multi-tensor shard: 290 segments, wd 0 on biases / LayerNorms."""
     segs = pythia_like_segments(layers, hidden, vocab)
     n = segs[-1][0] + segs[-1][1]
-    return Workload(f"pythia_{'1.4b' if layers == 24 else 'mini'}_shaped_fp16", n, grad_sigma=1e-4,
+    return Workload(f"pythia_1.4b_shaped_{layers}layer_fp16" if layers != 24 else "pythia_1.4b_shaped_fp16", n, grad_sigma=1e-4,
                     init_scale=2.0 ** 12, scale_window=1000, steps=10, segments=segs, cfg_id=1)
 
 
@@ -109,5 +109,12 @@ def opt_style_5b(numel=5_000_000_000) -> Workload:
                     scale_window=1000, lr=1.2e-4, clip=0.3, steps=100, inject_steps=(3, 4, 57), cfg_id=4)
 
 
+def pythia_2layer() -> Workload:
+    """The Pythia-1.4B layout cut to 2 layers (306,761,728 params, 4.9 GB of
+    state): the same kernels and segment kinds at a size that detailed
+    profiler captures handle."""
+    return pythia_1p4b(layers=2)
+
+
 ALL = {"tiny": tiny, "pythia_1p4b": pythia_1p4b, "neox20b_slice": neox20b_zero1_slice,
-       "accum8": accum8_predivide, "opt_5b": opt_style_5b}
+       "accum8": accum8_predivide, "opt_5b": opt_style_5b, "pythia_2layer": pythia_2layer}

@@ -1,0 +1,245 @@
+"""GPU parity at the workloads' full sizes, in the launch configuration bench.py
+times.
+
+Per step the oracle sees every gradient (copied to the host in chunks and
+passed through its single-threaded pass-1 routine on several host threads),
+so the overflow flag, the loss-scale trajectory and the norm are checked on
+the whole shard.  The AdamW state is tracked by the oracle on a deterministic
+sample of elements (every 4096th, the first and last 65,536, windows around
+2^31 and 2^32 and around segment boundaries): apart from the global norm and
+flag, each element's update depends only on its own inputs, so the sampled
+comparison is exact in what it checks.  Long traces (100 calls) are checked
+through properties that hold at any size: the flag equals "some input is not
+finite" (a sum of finite FP16/BF16 values cannot overflow FP32), and the scale
+follows the scaler rule.
+"""
+import os
+import time
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from mixed_precision_zero_b200 import Hparams, NeoxShard
+from synth import workloads as W
+from tests.gpu_harness import Guarded, check_close, check_ulp16
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+THREADS = max(1, len(os.sched_getaffinity(0)))
+
+
+def sample_indices(n, segments=None):
+    parts = [np.arange(0, n, 4096, dtype=np.int64), np.arange(0, min(n, 65536)), np.arange(max(0, n - 65536), n)]
+    for b in (1 << 31, 1 << 32):
+        if b < n:
+            parts.append(np.arange(max(0, b - 64), min(n, b + 64)))
+    for off, cnt, *_ in (segments or []):
+        parts.append(np.arange(max(0, off - 4), min(n, off + 4)))
+    return np.unique(np.concatenate(parts))
+
+
+class FullRun:
+    def __init__(self, wl: W.Workload, seed_offset=0):
+        self.wl = wl
+        n = wl.numel
+        dt = torch.bfloat16 if wl.bf16 else torch.float16
+        off = wl.elem_offset
+        self.seed = wl.seed + seed_offset
+        self.g = [Guarded(n, dt, off) for _ in range(wl.K)]
+        self.w = Guarded(n, dt, off)
+        self.master = Guarded(n, torch.float32, off)
+        self.m = Guarded(n, torch.float32, off)
+        self.v = Guarded(n, torch.float32, off)
+        synth.gpu_master_normal(self.master.t, wl.master_sigma, self.seed)
+        for so, sc, _, init in (wl.segments or []):
+            if init == "zero":
+                self.master.t[so:so + sc].zero_()
+            elif init == "one":
+                self.master.t[so:so + sc].fill_(1.0)
+        self.m.t.zero_()
+        self.v.t.zero_()
+        self.w.t.copy_(self.master.t.to(dt))
+        self.hp = Hparams(wl.beta1, wl.beta2, wl.eps, wl.clip, wl.predivide, wl.init_scale, 2.0, 1.0, wl.scale_window)
+        self.shard = NeoxShard(self.master.t, self.m.t, self.v.t, self.hp, wdtype=dt, gdtype=dt,
+                               segments=wl.seg_table(), weight_decay=wl.weight_decay, max_grads=wl.K)
+        self.ohp = oracle.OracleHparams(wl.beta1, wl.beta2, wl.eps, wl.clip, wl.predivide, wl.init_scale, 2.0, 1.0,
+                                        wl.scale_window)
+        self.scaler = oracle.Scaler(wl.init_scale, 0, 0)
+        self.segs = oracle.segments_array(wl.seg_table(), n, wl.weight_decay)
+        self.idx = sample_indices(n, wl.segments)
+        self.idx_dev = torch.from_numpy(self.idx).cuda()
+        self.s_master = self._gather32(self.master.t)
+        self.s_m = np.zeros_like(self.s_master)
+        self.s_v = np.zeros_like(self.s_master)
+        self.s_w = oracle.encode16(self.s_master, wl.bf16)
+        torch.cuda.synchronize()
+        self.n_inject = 0
+
+    def _gather32(self, t):
+        return t[self.idx_dev].cpu().numpy().copy()
+
+    def _gather16(self, t):
+        return t.view(torch.int16)[self.idx_dev].cpu().numpy().view(np.uint16).copy()
+
+    def gen(self, s):
+        wl = self.wl
+        for k, g in enumerate(self.g):
+            if wl.grad_dist == "t3":
+                synth.gpu_grad_t3_16(g.t, self.scaler.scale, self.seed, k, s, wl.bf16)
+            else:
+                synth.gpu_grad_normal16(g.t, wl.grad_sigma, self.scaler.scale, self.seed, k, s, wl.bf16)
+        if s in wl.inject_steps:
+            i = synth.inject_index(wl.numel, self.seed, s)
+            code = np.uint16(synth.inject_value(self.n_inject, wl.bf16)).view(np.int16)
+            self.g[0].t.view(torch.int16)[i] = int(code)
+            self.n_inject += 1
+        hits = 0
+        if s in wl.inject_rate_steps:
+            for k, g in enumerate(self.g):
+                hits += synth.gpu_rate_inject(g.t, wl.inject_rate, self.seed, k, s, wl.bf16)
+        return hits
+
+    def oracle_pass1(self, chunk=1 << 26):
+        """(non-finite count, sum of squares) over the whole shard on the host."""
+        wl = self.wl
+        inv_pre, inv_us = oracle.ingest_factors(wl.K, wl.predivide, self.scaler.scale)
+        n = wl.numel
+        bufs = [torch.empty(min(chunk, n), dtype=torch.int16, pin_memory=True) for _ in range(wl.K)]
+        bad, ssum = 0, 0.0
+        for lo in range(0, n, chunk):
+            hi = min(n, lo + chunk)
+            host = []
+            for g, b in zip(self.g, bufs):
+                b[: hi - lo].copy_(g.t.view(torch.int16)[lo:hi])
+                host.append(b[: hi - lo].numpy().view(np.uint16))
+            nb, s = oracle.grad_stats(host, wl.bf16, inv_pre, inv_us, threads=THREADS, chunk=1 << 22)
+            bad += nb
+            ssum += s
+        return bad, ssum
+
+    def step(self, s, check_state_every_step=False):
+        wl = self.wl
+        torch.cuda.synchronize()
+        nb, ssum = self.oracle_pass1()
+        sub = [self._gather16(g.t) for g in self.g]
+        res = self.shard.step([g.t for g in self.g], self.w.t, wl.lr)
+        info = oracle.step_decide(self.ohp, self.scaler, wl.lr, nb, ssum)
+        assert res.overflow == info.overflow, (s, res.overflow, info.overflow, nb)
+        assert res.loss_scale == info.scale_used and res.loss_scale_next == info.scale_next
+        assert res.applied_steps == info.t and res.good_steps == self.scaler.good
+        if not info.overflow:
+            assert abs(res.grad_norm - info.norm) <= 1e-5 * info.norm, (res.grad_norm, info.norm)
+            assert abs(res.clip_coef - info.coef) <= 1e-5 * info.coef
+            oracle.adam_apply(self.idx.astype(np.uint64), 0, sub, wl.bf16, self.segs, self.s_master, self.s_m,
+                              self.s_v, self.s_w, wl.bf16, self.ohp, wl.lr, info)
+        if check_state_every_step:
+            self.check_state()
+        return res, info, nb
+
+    def check_state(self):
+        check_close("master", self._gather32(self.master.t), self.s_master)
+        check_close("exp_avg", self._gather32(self.m.t), self.s_m)
+        check_close("exp_avg_sq", self._gather32(self.v.t), self.s_v)
+        check_ulp16(self._gather16(self.w.t), self.s_w)
+
+    def guards_intact(self):
+        return all(x.guards_intact() for x in (*self.g, self.w, self.master, self.m, self.v))
+
+    def close(self):
+        self.shard.close()
+        for x in (*self.g, self.w, self.master, self.m, self.v):
+            del x.base, x.t
+        torch.cuda.empty_cache()
+
+
+@pytest.fixture(autouse=True)
+def _free_memory():
+    torch.cuda.set_device(0)
+    yield
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+def _run(wl, steps, every=False):
+    t0 = time.time()
+    r = FullRun(wl)
+    flags = []
+    for s in range(1, steps + 1):
+        r.gen(s)
+        res, info, nb = r.step(s, check_state_every_step=every)
+        flags.append(res.overflow)
+    r.check_state()
+    assert r.guards_intact()
+    print(f"{wl.name}: {steps} steps, {len(r.idx)} sampled elements, {time.time() - t0:.1f}s, "
+          f"{THREADS} host threads")
+    return r, flags
+
+
+def test_pythia_1p4b_shaped_full_size():
+    wl = W.pythia_1p4b()
+    r, flags = _run(wl, 3, every=True)
+    assert flags == [0, 0, 0]
+    r.close()
+
+
+def test_neox20b_slice_misaligned_full_size():
+    """2,570,000,001 elements (> 2^31, odd) at element offset 3 of every array."""
+    wl = W.neox20b_zero1_slice()
+    r, flags = _run(wl, 3)
+    assert flags == [0, 0, 0]
+    r.close()
+
+
+def test_accum8_predivide_full_size():
+    """K = 8 Student-t(3) x 2^10 buffers: the natural FP16 overflows drive the
+    scale down until a step applies; the oracle's exact count of non-finite
+    inputs decides every flag."""
+    wl = W.accum8_predivide()
+    r, flags = _run(wl, 8)
+    assert flags[0] == 1 and flags[-1] == 0
+    r.close()
+
+
+def test_opt_style_5e9_bf16_full_size():
+    """5e9 BF16 elements (> 2^32), scripted overflows on calls 3 and 4."""
+    wl = W.opt_style_5b()
+    r, flags = _run(wl, 5)
+    assert flags == [0, 0, 1, 1, 0]
+    assert r.scaler.scale == 2.0 ** 14 and r.scaler.t == 3
+    r.close()
+
+
+def _trace_property(wl, steps):
+    """Full trace on the GPU; flags against 'some input not finite' (torch
+    reduction on the device) and the scale against the scaler rule."""
+    r = FullRun(wl)
+    scale, good, t = wl.init_scale, 0, 0
+    flags = []
+    for s in range(1, steps + 1):
+        r.scaler.scale = scale
+        hits = r.gen(s)
+        bad = any(not bool(torch.isfinite(g.t).all().item()) for g in r.g)
+        res = r.shard.step([g.t for g in r.g], r.w.t, wl.lr)
+        assert res.overflow == int(bad), (s, res.overflow, bad, hits)
+        scale, good, t = oracle.scaler_update(r.ohp, scale, good, t, bad)
+        if not bad:
+            t += 1
+        assert res.loss_scale_next == scale and res.applied_steps == t and res.good_steps == good
+        flags.append(res.overflow)
+    r.close()
+    return flags, scale, t
+
+
+def test_opt_style_100_call_trace():
+    flags, scale, t = _trace_property(W.opt_style_5b(), 100)
+    assert [i + 1 for i, f in enumerate(flags) if f] == [3, 4, 57]
+    assert scale == 2.0 ** 13 and t == 97
+
+
+def test_accum8_30_call_trace():
+    flags, scale, t = _trace_property(W.accum8_predivide(), 30)
+    assert flags[0] == 1 and 0 in flags
+    assert flags[19] == 1 and flags[24] == 1  # rate injections on calls 20 and 25
