@@ -142,6 +142,28 @@ neox_status neox_shard_create(const neox_shard_desc* desc, const neox_hparams* h
 neox_status neox_shard_step(neox_shard* h, const void* const* grads, int32_t num_grads,
                             void* params, float lr, void* cuda_stream, neox_step_result* out);
 
+/* The same step, enqueued on cuda_stream without waiting for it, so that a
+ * training loop never blocks on the optimizer and a CUDA graph can capture it.
+ * The differences from neox_shard_step:
+ *   - nothing is read back to the host: the GPU writes the step's result into
+ *     `result` (device memory or pinned host memory the caller owns, 8-byte
+ *     aligned; NULL = not written) when pass 1 finishes;
+ *   - the bias corrections bc1 = 1-b1^t, bc2 = 1-b2^t are formed on the GPU
+ *     in double from the device copy of t (pow in double; the synchronous
+ *     step forms them on the host), so the state agrees with the synchronous
+ *     step within the step's tolerances rather than bit for bit;
+ *   - when lr_device is non-NULL the learning rate is read from that device
+ *     float at run time (a captured graph can then change it without
+ *     re-capture) and `lr` is ignored;
+ *   - profiling events are not recorded (launches are still counted).
+ * It launches only kernels (no allocation, copy or synchronisation), so it can
+ * be captured into a CUDA graph once the handle has run one step outside a
+ * capture.  The arrays and `result` must stay valid until the step finishes.
+ * After asynchronous steps, neox_shard_get_state / neox_shard_step /
+ * neox_shard_set_state first wait for the last stream used here. */
+neox_status neox_shard_step_async(neox_shard* h, const void* const* grads, int32_t num_grads, void* params,
+                                  float lr, const float* lr_device, void* cuda_stream, neox_step_result* result);
+
 /* Replace the hyperparameters (e.g. the clip 1.0 -> 0.3 change); the current
  * loss scale and counters are kept (init_scale is ignored here). */
 neox_status neox_shard_set_hparams(neox_shard* h, const neox_hparams* hp);

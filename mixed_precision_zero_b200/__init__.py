@@ -21,7 +21,7 @@ from ._abi import (NEOX_BF16, NEOX_ERR_CUDA, NEOX_ERR_INVALID_ARGUMENT, NEOX_ERR
                    neox_shard_create, neox_shard_desc, neox_shard_destroy, neox_shard_get_profile,
                    neox_shard_get_state, neox_shard_reset_profile, neox_shard_scratch_bytes,
                    neox_shard_set_hparams, neox_shard_set_profiling, neox_shard_set_state,
-                   neox_shard_step, neox_status_string, neox_step_result)
+                   neox_shard_step, neox_shard_step_async, neox_status_string, neox_step_result)
 
 __all__ = ["NeoxShard", "Hparams", "NeoxError", "neox_shard_create", "neox_shard_step",
            "neox_shard_destroy", "neox_shard_set_hparams", "neox_shard_get_state",
@@ -85,17 +85,33 @@ class NeoxShard:
             self.device = torch.cuda.current_device()
         self.handle = neox_shard_create(desc, hp.c(), self.device)
 
-    def step(self, grads, params, lr: float, stream=None) -> neox_step_result:
-        import torch
+    def _check(self, grads, params):
         for g in grads:
             if g.numel() != self.numel or _dtype_code(g) != self.gdtype or not g.is_contiguous():
                 raise ValueError("each grad must be a contiguous 16-bit tensor of the shard's gradient type and length")
         if params.numel() != self.numel or _dtype_code(params) != self.wdtype or not params.is_contiguous():
             raise ValueError("params must be a contiguous 16-bit tensor of the shard's weight type and length")
+
+    def step(self, grads, params, lr: float, stream=None) -> neox_step_result:
+        import torch
+        self._check(grads, params)
         if stream is None:
             stream = torch.cuda.current_stream(self.device)
         sp = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
         return neox_shard_step(self.handle, [g.data_ptr() for g in grads], params.data_ptr(), lr, sp)
+
+    def step_async(self, grads, params, lr: float = 0.0, *, result=None, lr_device=None, stream=None) -> None:
+        """Enqueue a step without waiting.  `result`: a device (or pinned) tensor
+        of at least 32 bytes that receives the neox_step_result; `lr_device`: a
+        float32 CUDA tensor holding the learning rate (read at run time)."""
+        import torch
+        self._check(grads, params)
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device)
+        sp = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+        neox_shard_step_async(self.handle, [g.data_ptr() for g in grads], params.data_ptr(), lr, sp,
+                              None if result is None else result.data_ptr(),
+                              None if lr_device is None else lr_device.data_ptr())
 
     def set_hparams(self, hp: Hparams) -> None:
         neox_shard_set_hparams(self.handle, hp.c())

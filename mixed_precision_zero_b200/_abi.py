@@ -78,6 +78,9 @@ def lib() -> ctypes.CDLL:
         L.neox_shard_step.argtypes = [_H, ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32, ctypes.c_void_p,
                                       ctypes.c_float, ctypes.c_void_p, ctypes.POINTER(neox_step_result)]
         L.neox_shard_step.restype = S
+        L.neox_shard_step_async.argtypes = [_H, ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32, ctypes.c_void_p,
+                                            ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+        L.neox_shard_step_async.restype = S
         L.neox_shard_set_hparams.argtypes = [_H, ctypes.POINTER(neox_hparams)]
         L.neox_shard_set_hparams.restype = S
         L.neox_shard_get_state.argtypes = [_H, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int32),
@@ -135,6 +138,14 @@ def neox_shard_step(h: int, grad_ptrs, params_ptr: int, lr: float, stream: int) 
     if st != NEOX_OK:
         raise NeoxError(st, lib().neox_last_error(h).decode())
     return res
+
+
+def neox_shard_step_async(h: int, grad_ptrs, params_ptr: int, lr: float, stream: int,
+                          result_ptr: int | None = None, lr_device_ptr: int | None = None) -> None:
+    arr = (ctypes.c_void_p * len(grad_ptrs))(*grad_ptrs)
+    st = lib().neox_shard_step_async(h, arr, len(grad_ptrs), params_ptr, lr, lr_device_ptr, stream, result_ptr)
+    if st != NEOX_OK:
+        raise NeoxError(st, lib().neox_last_error(h).decode())
 
 
 def neox_shard_set_hparams(h: int, hp: neox_hparams) -> None:

@@ -68,7 +68,10 @@ struct __align__(64) DevScalars {
     float scale_used;      // S the last step's grads carried
     float norm;            // pre-clip norm of the last step (+inf on overflow)
     unsigned int blocks_done;  // pass-1 ticket counter, back to 0 after each step
-    int32_t pad_[5];
+    float step_size;       // device-computed fl32(lr / bc1) of the last step (asynchronous steps)
+    float bc2_sqrt;        // device-computed fl32(sqrt(bc2)) of the last step (asynchronous steps)
+    float lr;              // learning rate of the last step (asynchronous steps)
+    int32_t pad_[2];
 };
 static_assert(sizeof(DevScalars) == 64, "DevScalars is one 64-byte block");
 
@@ -84,6 +87,12 @@ struct ScalerArgs {
     float clip;           // <= 0: off
     float factor, min_scale;
     int32_t window;
+    // asynchronous steps: the bias corrections are formed on the device from
+    // the device step count, and the result is written to `result`
+    int32_t device_bc;
+    float lr, beta1, beta2;
+    const float* lr_ptr;       // when non-NULL, the learning rate is read here
+    neox_step_result* result;  // device-accessible; NULL = not written
 };
 
 struct AdamArgs {
@@ -91,6 +100,7 @@ struct AdamArgs {
     float step_size;      // fl32(lr / bc1) for t+1
     float bcs;            // fl32(sqrt(bc2)) for t+1
     float inv_pre;
+    int32_t device_bc;    // take lr, step_size and bcs from the device scalars
     double post;
 };
 
@@ -318,6 +328,10 @@ grad_stats_kernel(GradPtrs gp, int K, Layout L, ScalerArgs sa, float* __restrict
         }
     }
 
+    // Let the update kernel's blocks start their prologue as this grid winds
+    // down; they wait (griddepcontrol.wait) for this grid's completion before
+    // reading anything it writes.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     block_reduce<kThreads1>(s, bad, sh_s, sh_b);
     if (threadIdx.x == 0) {
         part_s[blockIdx.x] = s;
@@ -377,6 +391,26 @@ grad_stats_kernel(GradPtrs gp, int K, Layout L, ScalerArgs sa, float* __restrict
     sc->scale = S;
     sc->good = good;
     sc->t = t;
+    if (sa.device_bc) {
+        const float lr = sa.lr_ptr ? *sa.lr_ptr : sa.lr;
+        sc->lr = lr;
+        if (!overflow) {
+            const double bc1 = 1.0 - pow((double)sa.beta1, (double)t);
+            const double bc2 = 1.0 - pow((double)sa.beta2, (double)t);
+            sc->step_size = (float)((double)lr / bc1);
+            sc->bc2_sqrt = (float)sqrt(bc2);
+        }
+        if (sa.result) {
+            neox_step_result* r = sa.result;
+            r->overflow = overflow;
+            r->grad_norm = sc->norm;
+            r->clip_coef = sc->coef;
+            r->loss_scale = sc->scale_used;
+            r->loss_scale_next = S;
+            r->good_steps = good;
+            r->applied_steps = t;
+        }
+    }
     sc->blocks_done = 0;
 }
 
@@ -421,13 +455,21 @@ __device__ __forceinline__ void adam_vec(const float (&g)[VEC], const float (&ke
 
 template <class G, class W, int VEC, bool READ_ACC>
 __global__ void __launch_bounds__(kThreads3)
-adam_kernel(GradPtrs gp, int K, const float* __restrict__ acc, Layout L, AdamArgs a,
+adam_kernel(GradPtrs gp, int K, const float* __restrict__ acc, Layout L, AdamArgs a_arg,
             float* __restrict__ master, float* __restrict__ m, float* __restrict__ v, uint16_t* __restrict__ w,
             const unsigned long long* __restrict__ seg_end, const float* __restrict__ seg_wd, int nsegs,
             const DevScalars* __restrict__ sc) {
+    // Programmatic dependent launch: everything below reads what pass 1 wrote.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     if (sc->overflow) return;  // skipped step: nothing is written
     const float c = sc->coef;
+    AdamArgs a = a_arg;
     const float inv_us = unscale_factor(a.post, sc->scale_used);
+    if (a.device_bc) {
+        a.lr = sc->lr;
+        a.step_size = sc->step_size;
+        a.bcs = sc->bc2_sqrt;
+    }
 
     const unsigned long long stride = (unsigned long long)gridDim.x * kThreads3;
     unsigned long long v0 = (unsigned long long)blockIdx.x * kThreads3 + threadIdx.x;
@@ -551,6 +593,8 @@ struct neox_shard {
     unsigned long long owned_bytes = 0;
     // profiling
     bool profiling = false;
+    bool mirror_stale = false;        // asynchronous steps ran since the last read
+    cudaStream_t last_stream = nullptr;
     cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};
     neox_profile prof{};
     std::string last_error;
@@ -664,9 +708,21 @@ cudaError_t launch_pass2(neox_shard* h, const GradPtrs& gp, int K, const float* 
                          const AdamArgs& a, uint16_t* w, cudaStream_t st) {
     auto kern = adam_kernel<G, W, VEC, ACC>;
     const int grid = grid_for(kern, kThreads3, L.nvec, h->sm_count, 1 << 20);
-    kern<<<grid, kThreads3, 0, st>>>(gp, K, acc, L, a, h->master, h->m, h->v, w, h->d_seg_end, h->d_seg_wd,
-                                     h->nsegs, h->d_sc);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads3);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const float* accp = acc;
+    const unsigned long long* se = h->d_seg_end;
+    const float* sw = h->d_seg_wd;
+    const DevScalars* sc = h->d_sc;
+    return cudaLaunchKernelEx(&cfg, kern, gp, K, accp, L, a, h->master, h->m, h->v, w, se, sw, h->nsegs, sc);
 }
 
 template <class G, int VEC>
@@ -715,6 +771,114 @@ void free_all(neox_shard* h) {
     if (h->h_sc) cudaFreeHost(h->h_sc);
     for (auto& e : h->ev)
         if (e) cudaEventDestroy(e);
+}
+
+// Bring the host copy of the scaler state up to date after asynchronous steps.
+neox_status refresh_mirror(neox_shard* h) {
+    if (!h->mirror_stale) return NEOX_OK;
+    DeviceGuard g(h->device);
+    cudaError_t e;
+    if ((e = cudaStreamSynchronize(h->last_stream)) != cudaSuccess) return cuda_fail(h, e, "waiting for asynchronous steps");
+    DevScalars r;
+    if ((e = cudaMemcpy(&r, h->d_sc, sizeof(r), cudaMemcpyDeviceToHost)) != cudaSuccess)
+        return cuda_fail(h, e, "reading the device scaler state");
+    h->scale = r.scale;
+    h->good = r.good;
+    h->t = r.t;
+    h->mirror_stale = false;
+    return NEOX_OK;
+}
+
+// Validate the arguments of a step and enqueue its two kernels on `st`.
+// device_bc = false: bias corrections from the host copy of t (synchronous
+// steps, whose caller keeps that copy current).  device_bc = true: the last
+// pass-1 block forms them from the device step count and writes `result`.
+neox_status enqueue_step(neox_shard* h, const void* const* grads, int32_t num_grads, void* params, float lr,
+                         const float* lr_dev, cudaStream_t st, bool device_bc, neox_step_result* result) {
+    if (num_grads < 1 || num_grads > kMaxGrads) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "num_grads must be in [1, 64]");
+    if (!grads) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "grads is NULL");
+    if (!lr_dev && (!finite(lr) || lr < 0.0f)) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "lr must be finite and >= 0");
+    GradPtrs gp{};
+    uintptr_t a16[kMaxGrads + 1];
+    if (h->numel > 0) {
+        if (!params) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "params is NULL");
+        if ((uintptr_t)params & 1u) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "params must be 2-byte aligned");
+        for (int k = 0; k < num_grads; k++) {
+            if (!grads[k]) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "grads[" + std::to_string(k) + "] is NULL");
+            if ((uintptr_t)grads[k] & 1u)
+                return fail(h, NEOX_ERR_INVALID_ARGUMENT, "grads[" + std::to_string(k) + "] must be 2-byte aligned");
+            gp.p[k] = static_cast<const uint16_t*>(grads[k]);
+            a16[k] = (uintptr_t)grads[k];
+        }
+        a16[num_grads] = (uintptr_t)params;
+    }
+    if (result && ((uintptr_t)result & 7u)) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "result must be 8-byte aligned");
+    if (lr_dev && ((uintptr_t)lr_dev & 3u)) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "lr_device must be 4-byte aligned");
+
+    const bool use_acc = num_grads >= 5 && h->d_acc != nullptr;
+    uintptr_t a32[3] = {(uintptr_t)h->master, (uintptr_t)h->m, (uintptr_t)h->v};
+    int vec = 1;
+    Layout L = h->numel > 0 ? choose_layout(h->numel, a16, num_grads + 1, a32, 3, vec) : Layout{0, 0, 0, 0};
+    float* acc = nullptr;
+    if (use_acc) {
+        const unsigned long long hh = L.head % 4;
+        acc = h->d_acc + ((4 - hh) % 4);  // &acc[head] is 16-byte aligned
+    }
+
+    ScalerArgs sa{};
+    sa.post = (double)num_grads / (double)h->hp.predivide;
+    sa.inv_pre = (float)(1.0 / (double)h->hp.predivide);
+    sa.clip = h->hp.clip_norm;
+    sa.factor = h->hp.scale_factor;
+    sa.min_scale = h->hp.min_scale;
+    sa.window = h->hp.scale_window;
+    sa.device_bc = device_bc ? 1 : 0;
+    sa.lr = lr;
+    sa.beta1 = h->hp.beta1;
+    sa.beta2 = h->hp.beta2;
+    sa.lr_ptr = lr_dev;
+    sa.result = result;
+
+    AdamArgs a{};
+    a.lr = lr;
+    a.b1 = h->hp.beta1;
+    a.b2 = h->hp.beta2;
+    a.omb1 = 1.0f - h->hp.beta1;
+    a.omb2 = 1.0f - h->hp.beta2;
+    a.eps = h->hp.eps;
+    if (!device_bc) {
+        const double t1 = (double)(h->t + 1);  // the step count if this step is applied
+        const double bc1 = 1.0 - std::pow((double)h->hp.beta1, t1);
+        const double bc2 = 1.0 - std::pow((double)h->hp.beta2, t1);
+        a.step_size = (float)((double)lr / bc1);
+        a.bcs = (float)std::sqrt(bc2);
+    }
+    a.device_bc = device_bc ? 1 : 0;
+    a.inv_pre = sa.inv_pre;
+    a.post = sa.post;
+
+    const bool timed = h->profiling && !device_bc;
+    cudaError_t e;
+    if (timed && (e = cudaEventRecord(h->ev[0], st)) != cudaSuccess) return cuda_fail(h, e, "cudaEventRecord");
+    if (h->gdtype == NEOX_FP16) e = dispatch1v<F16>(h, vec, gp, num_grads, L, sa, acc, st);
+    else e = dispatch1v<BF16>(h, vec, gp, num_grads, L, sa, acc, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "pass-1 launch");
+    h->prof.launches += 1;
+    if (timed && (e = cudaEventRecord(h->ev[1], st)) != cudaSuccess) return cuda_fail(h, e, "cudaEventRecord");
+    if (h->numel > 0) {
+        uint16_t* w = static_cast<uint16_t*>(params);
+        if (h->gdtype == NEOX_FP16) {
+            e = h->wdtype == NEOX_FP16 ? dispatch2v<F16, F16>(h, vec, gp, num_grads, acc, L, a, w, st)
+                                       : dispatch2v<F16, BF16>(h, vec, gp, num_grads, acc, L, a, w, st);
+        } else {
+            e = h->wdtype == NEOX_FP16 ? dispatch2v<BF16, F16>(h, vec, gp, num_grads, acc, L, a, w, st)
+                                       : dispatch2v<BF16, BF16>(h, vec, gp, num_grads, acc, L, a, w, st);
+        }
+        if (e != cudaSuccess) return cuda_fail(h, e, "pass-2 launch");
+        h->prof.launches += 1;
+    }
+    if (timed && (e = cudaEventRecord(h->ev[2], st)) != cudaSuccess) return cuda_fail(h, e, "cudaEventRecord");
+    return NEOX_OK;
 }
 
 }  // namespace
@@ -876,6 +1040,7 @@ neox_status neox_shard_set_hparams(neox_shard* h, const neox_hparams* hp) {
 
 neox_status neox_shard_get_state(const neox_shard* h, float* scale, int32_t* good, int64_t* t) {
     if (!h) return NEOX_ERR_INVALID_ARGUMENT;
+    if (neox_status s = refresh_mirror(const_cast<neox_shard*>(h)); s != NEOX_OK) return s;
     if (scale) *scale = h->scale;
     if (good) *good = h->good;
     if (t) *t = h->t;
@@ -887,6 +1052,11 @@ neox_status neox_shard_set_state(neox_shard* h, float scale, int32_t good, int64
     if (!(scale > 0.0f) || !finite(scale) || good < 0 || t < 0)
         return fail(h, NEOX_ERR_INVALID_ARGUMENT, "state needs a finite scale > 0, good >= 0, t >= 0");
     DeviceGuard g(h->device);
+    if (h->mirror_stale) {
+        cudaError_t e0 = cudaStreamSynchronize(h->last_stream);
+        if (e0 != cudaSuccess) return cuda_fail(h, e0, "waiting for asynchronous steps");
+        h->mirror_stale = false;
+    }
     DevScalars s{};
     s.scale = scale;
     s.scale_used = scale;
@@ -925,82 +1095,14 @@ neox_status neox_shard_step(neox_shard* h, const void* const* grads, int32_t num
     if (!h) return NEOX_ERR_INVALID_ARGUMENT;
     h->last_error.clear();
     if (!out) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "out is NULL");
-    if (num_grads < 1 || num_grads > kMaxGrads) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "num_grads must be in [1, 64]");
-    if (!grads) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "grads is NULL");
-    if (!finite(lr) || lr < 0.0f) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "lr must be finite and >= 0");
-    GradPtrs gp{};
-    uintptr_t a16[kMaxGrads + 1];
-    if (h->numel > 0) {
-        if (!params) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "params is NULL");
-        if ((uintptr_t)params & 1u) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "params must be 2-byte aligned");
-        for (int k = 0; k < num_grads; k++) {
-            if (!grads[k]) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "grads[" + std::to_string(k) + "] is NULL");
-            if ((uintptr_t)grads[k] & 1u)
-                return fail(h, NEOX_ERR_INVALID_ARGUMENT, "grads[" + std::to_string(k) + "] must be 2-byte aligned");
-            gp.p[k] = static_cast<const uint16_t*>(grads[k]);
-            a16[k] = (uintptr_t)grads[k];
-        }
-        a16[num_grads] = (uintptr_t)params;
-    }
+    if (neox_status s = refresh_mirror(h); s != NEOX_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
     DeviceGuard g(h->device);
     if (!g.ok) return fail(h, NEOX_ERR_CUDA, "cudaSetDevice failed");
-    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
-
-    const bool use_acc = num_grads >= 5 && h->d_acc != nullptr;
-    uintptr_t a32[3] = {(uintptr_t)h->master, (uintptr_t)h->m, (uintptr_t)h->v};
-    int vec = 1;
-    Layout L = h->numel > 0 ? choose_layout(h->numel, a16, num_grads + 1, a32, 3, vec) : Layout{0, 0, 0, 0};
-    float* acc = nullptr;
-    if (use_acc) {
-        const unsigned long long hh = L.head % 4;
-        acc = h->d_acc + ((4 - hh) % 4);  // &acc[head] is 16-byte aligned
-    }
-
-    ScalerArgs sa;
-    sa.post = (double)num_grads / (double)h->hp.predivide;
-    sa.inv_pre = (float)(1.0 / (double)h->hp.predivide);
-    sa.clip = h->hp.clip_norm;
-    sa.factor = h->hp.scale_factor;
-    sa.min_scale = h->hp.min_scale;
-    sa.window = h->hp.scale_window;
-
-    AdamArgs a;
-    a.lr = lr;
-    a.b1 = h->hp.beta1;
-    a.b2 = h->hp.beta2;
-    a.omb1 = 1.0f - h->hp.beta1;
-    a.omb2 = 1.0f - h->hp.beta2;
-    a.eps = h->hp.eps;
-    {
-        const double t1 = (double)(h->t + 1);  // the step count if this step is applied
-        const double bc1 = 1.0 - std::pow((double)h->hp.beta1, t1);
-        const double bc2 = 1.0 - std::pow((double)h->hp.beta2, t1);
-        a.step_size = (float)((double)lr / bc1);
-        a.bcs = (float)std::sqrt(bc2);
-    }
-    a.inv_pre = sa.inv_pre;
-    a.post = sa.post;
-
+    const int64_t launches0 = h->prof.launches;
+    if (neox_status s = enqueue_step(h, grads, num_grads, params, lr, nullptr, st, false, nullptr); s != NEOX_OK)
+        return s;
     cudaError_t e;
-    if (h->profiling && (e = cudaEventRecord(h->ev[0], st)) != cudaSuccess) return cuda_fail(h, e, "cudaEventRecord");
-    if (h->gdtype == NEOX_FP16) e = dispatch1v<F16>(h, vec, gp, num_grads, L, sa, acc, st);
-    else e = dispatch1v<BF16>(h, vec, gp, num_grads, L, sa, acc, st);
-    if (e != cudaSuccess) return cuda_fail(h, e, "pass-1 launch");
-    h->prof.launches += 1;
-    if (h->profiling && (e = cudaEventRecord(h->ev[1], st)) != cudaSuccess) return cuda_fail(h, e, "cudaEventRecord");
-    if (h->numel > 0) {
-        uint16_t* w = static_cast<uint16_t*>(params);
-        if (h->gdtype == NEOX_FP16) {
-            e = h->wdtype == NEOX_FP16 ? dispatch2v<F16, F16>(h, vec, gp, num_grads, acc, L, a, w, st)
-                                       : dispatch2v<F16, BF16>(h, vec, gp, num_grads, acc, L, a, w, st);
-        } else {
-            e = h->wdtype == NEOX_FP16 ? dispatch2v<BF16, F16>(h, vec, gp, num_grads, acc, L, a, w, st)
-                                       : dispatch2v<BF16, BF16>(h, vec, gp, num_grads, acc, L, a, w, st);
-        }
-        if (e != cudaSuccess) return cuda_fail(h, e, "pass-2 launch");
-        h->prof.launches += 1;
-    }
-    if (h->profiling && (e = cudaEventRecord(h->ev[2], st)) != cudaSuccess) return cuda_fail(h, e, "cudaEventRecord");
     if ((e = cudaMemcpyAsync(h->h_sc, h->d_sc, sizeof(DevScalars), cudaMemcpyDeviceToHost, st)) != cudaSuccess)
         return cuda_fail(h, e, "cudaMemcpyAsync result");
     if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(h, e, "step execution");
@@ -1027,6 +1129,21 @@ neox_status neox_shard_step(neox_shard* h, const void* const* grads, int32_t num
         h->prof.last_grad_pass_ms = t01;
         h->prof.last_update_pass_ms = t12;
     }
+    (void)launches0;
+    return NEOX_OK;
+}
+
+neox_status neox_shard_step_async(neox_shard* h, const void* const* grads, int32_t num_grads, void* params,
+                                  float lr, const float* lr_device, void* cuda_stream, neox_step_result* result) {
+    if (!h) return NEOX_ERR_INVALID_ARGUMENT;
+    h->last_error.clear();
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    DeviceGuard g(h->device);
+    if (!g.ok) return fail(h, NEOX_ERR_CUDA, "cudaSetDevice failed");
+    if (neox_status s = enqueue_step(h, grads, num_grads, params, lr, lr_device, st, true, result); s != NEOX_OK)
+        return s;
+    h->mirror_stale = true;
+    h->last_stream = st;
     return NEOX_OK;
 }
 
@@ -1205,14 +1322,14 @@ neox_status neox_shard_step_noalloc(const neox_shard_desc* d, const neox_hparams
     int vec = 1;
     Layout L = d->numel > 0 ? choose_layout(d->numel, a16, num_grads + 1, a32, 3, vec) : Layout{0, 0, 0, 0};
 
-    ScalerArgs sa;
+    ScalerArgs sa{};
     sa.post = (double)num_grads / (double)hp->predivide;
     sa.inv_pre = (float)(1.0 / (double)hp->predivide);
     sa.clip = hp->clip_norm;
     sa.factor = hp->scale_factor;
     sa.min_scale = hp->min_scale;
     sa.window = hp->scale_window;
-    AdamArgs a;
+    AdamArgs a{};
     a.lr = lr;
     a.b1 = hp->beta1;
     a.b2 = hp->beta2;
