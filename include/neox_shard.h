@@ -159,8 +159,11 @@ neox_status neox_shard_step(neox_shard* h, const void* const* grads, int32_t num
  * It launches only kernels (no allocation, copy or synchronisation), so it can
  * be captured into a CUDA graph once the handle has run one step outside a
  * capture.  The arrays and `result` must stay valid until the step finishes.
- * After asynchronous steps, neox_shard_get_state / neox_shard_step /
- * neox_shard_set_state first wait for the last stream used here. */
+ * Once a handle has issued an asynchronous step (whose graph replays the
+ * library cannot see), its scaler state lives on the device only:
+ * neox_shard_get_state and neox_shard_set_state then wait for the whole
+ * device (cudaDeviceSynchronize) and read or write the device copy, and
+ * neox_shard_step forms its bias corrections on the device as well. */
 neox_status neox_shard_step_async(neox_shard* h, const void* const* grads, int32_t num_grads, void* params,
                                   float lr, const float* lr_device, void* cuda_stream, neox_step_result* result);
 

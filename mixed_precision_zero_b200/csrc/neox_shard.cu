@@ -199,11 +199,17 @@ __device__ __forceinline__ void ingest(const GradPtrs& gp, int K, unsigned long 
                                        float inv_pre, float inv_us, float (&g)[VEC]) {
 #pragma unroll
     for (int e = 0; e < VEC; e++) g[e] = 0.0f;
+    const bool pre1 = inv_pre == 1.0f;  // x * 1 == x exactly: skip the multiply
     for (int k = 0; k < K; k++) {
         uint16_t h[VEC];
         ld16<VEC>(gp.p[k] + i, h);
+        if (pre1) {
 #pragma unroll
-        for (int e = 0; e < VEC; e++) g[e] = __fadd_rn(g[e], __fmul_rn(G::dec(h[e]), inv_pre));
+            for (int e = 0; e < VEC; e++) g[e] = __fadd_rn(g[e], G::dec(h[e]));
+        } else {
+#pragma unroll
+            for (int e = 0; e < VEC; e++) g[e] = __fadd_rn(g[e], __fmul_rn(G::dec(h[e]), inv_pre));
+        }
     }
 #pragma unroll
     for (int e = 0; e < VEC; e++) g[e] = __fmul_rn(g[e], inv_us);
@@ -220,14 +226,22 @@ __device__ __forceinline__ void ingest_batch(const GradPtrs& gp, int K, unsigned
     for (int u = 0; u < U; u++)
 #pragma unroll
         for (int e = 0; e < VEC; e++) g[u][e] = 0.0f;
+    const bool pre1 = inv_pre == 1.0f;  // x * 1 == x exactly: skip the multiply
     for (int k = 0; k < K; k++) {
         uint16_t h[U][VEC];
 #pragma unroll
         for (int u = 0; u < U; u++) ld16<VEC>(gp.p[k] + i0 + u * di, h[u]);
+        if (pre1) {
 #pragma unroll
-        for (int u = 0; u < U; u++)
+            for (int u = 0; u < U; u++)
 #pragma unroll
-            for (int e = 0; e < VEC; e++) g[u][e] = __fadd_rn(g[u][e], __fmul_rn(G::dec(h[u][e]), inv_pre));
+                for (int e = 0; e < VEC; e++) g[u][e] = __fadd_rn(g[u][e], G::dec(h[u][e]));
+        } else {
+#pragma unroll
+            for (int u = 0; u < U; u++)
+#pragma unroll
+                for (int e = 0; e < VEC; e++) g[u][e] = __fadd_rn(g[u][e], __fmul_rn(G::dec(h[u][e]), inv_pre));
+        }
     }
 #pragma unroll
     for (int u = 0; u < U; u++)
@@ -239,23 +253,27 @@ __device__ __forceinline__ float unscale_factor(double post, float scale) {
     return (float)(1.0 / (post * (double)scale));
 }
 
-// Sum of squares of a vector: FP32 within the vector, recomputed in FP64 in
-// the (degenerate) case that a finite element squares past FP32's range.
+// Sum of squares of a vector (FP32 within the vector) and the non-finite
+// flag.  A sum of squares is finite exactly when every element is finite and
+// no square or partial sum passes FP32's range, so one test per vector
+// replaces a test per element; only a vector that fails it looks at its
+// elements (and, when they are all finite, redoes the sum in FP64).
 template <int VEC>
 __device__ __forceinline__ double vec_sumsq(const float (&g)[VEC], int& bad) {
     float q = 0.0f;
-    int vb = 0;
 #pragma unroll
-    for (int e = 0; e < VEC; e++) {
-        vb |= not_finite(g[e]);
-        q = __fmaf_rn(g[e], g[e], q);
-    }
-    bad |= vb;
-    if (!vb && not_finite(q)) {
-        double d = 0.0;
+    for (int e = 0; e < VEC; e++) q = __fmaf_rn(g[e], g[e], q);
+    if (!(q <= 3.40282346638528859812e+38f)) {
+        int vb = 0;
 #pragma unroll
-        for (int e = 0; e < VEC; e++) d += (double)g[e] * (double)g[e];
-        return d;
+        for (int e = 0; e < VEC; e++) vb |= not_finite(g[e]);
+        bad |= vb;
+        if (!vb) {
+            double d = 0.0;
+#pragma unroll
+            for (int e = 0; e < VEC; e++) d += (double)g[e] * (double)g[e];
+            return d;
+        }
     }
     return (double)q;
 }
@@ -285,8 +303,39 @@ __device__ __forceinline__ void block_reduce(double& s, int& bad, double* sh_s, 
 }
 
 // ---------------------------------------------------------------- pass 1
+// The vector loop of pass 1.  KFIX = 1 compiles the single-buffer case with
+// K known to be 1; KFIX = 0 takes K at run time.
+template <class G, int VEC, bool WRITE_ACC, int KFIX>
+__device__ __forceinline__ void pass1_vectors(const GradPtrs& gp, int K_rt, const Layout& L, float inv_pre,
+                                              float inv_us, float* __restrict__ acc, double& s, int& bad) {
+    const int K = KFIX ? KFIX : K_rt;
+    // Several buffers already give several loads in flight per vector: a
+    // shorter unroll keeps that variant within its registers.
+    constexpr int U = KFIX ? kUnroll1 : 2;
+    // Grid-stride over vectors, U strides per iteration (the thread still
+    // visits its vectors in the same order, so its sum is unchanged).
+    const unsigned long long stride = (unsigned long long)gridDim.x * kThreads1;
+    unsigned long long v = (unsigned long long)blockIdx.x * kThreads1 + threadIdx.x;
+    for (; v + (U - 1) * stride < L.nvec; v += U * stride) {
+        float g[U][VEC];
+        ingest_batch<G, VEC, U>(gp, K, L.head + v * VEC, stride * VEC, inv_pre, inv_us, g);
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+            s += vec_sumsq<VEC>(g[u], bad);
+            if constexpr (WRITE_ACC) st32<VEC>(acc + L.head + (v + u * stride) * VEC, g[u]);
+        }
+    }
+    for (; v < L.nvec; v += stride) {
+        const unsigned long long i = L.head + v * VEC;
+        float g[VEC];
+        ingest<G, VEC>(gp, K, i, inv_pre, inv_us, g);
+        s += vec_sumsq<VEC>(g, bad);
+        if constexpr (WRITE_ACC) st32<VEC>(acc + i, g);
+    }
+}
+
 template <class G, int VEC, bool WRITE_ACC>
-__global__ void __launch_bounds__(kThreads1)
+__global__ void __launch_bounds__(kThreads1, 1024 / kThreads1)
 grad_stats_kernel(GradPtrs gp, int K, Layout L, ScalerArgs sa, float* __restrict__ acc,
                   double* __restrict__ part_s, int* __restrict__ part_b, DevScalars* __restrict__ sc) {
     __shared__ double sh_s[kThreads1 / 32];
@@ -297,26 +346,8 @@ grad_stats_kernel(GradPtrs gp, int K, Layout L, ScalerArgs sa, float* __restrict
     double s = 0.0;
     int bad = 0;
 
-    // Grid-stride over vectors, kUnroll1 strides per iteration (the thread
-    // still visits its vectors in the same order, so its sum is unchanged).
-    const unsigned long long stride = (unsigned long long)gridDim.x * kThreads1;
-    unsigned long long v = (unsigned long long)blockIdx.x * kThreads1 + threadIdx.x;
-    for (; v + (kUnroll1 - 1) * stride < L.nvec; v += kUnroll1 * stride) {
-        float g[kUnroll1][VEC];
-        ingest_batch<G, VEC, kUnroll1>(gp, K, L.head + v * VEC, stride * VEC, sa.inv_pre, inv_us, g);
-#pragma unroll
-        for (int u = 0; u < kUnroll1; u++) {
-            s += vec_sumsq<VEC>(g[u], bad);
-            if constexpr (WRITE_ACC) st32<VEC>(acc + L.head + (v + u * stride) * VEC, g[u]);
-        }
-    }
-    for (; v < L.nvec; v += stride) {
-        const unsigned long long i = L.head + v * VEC;
-        float g[VEC];
-        ingest<G, VEC>(gp, K, i, sa.inv_pre, inv_us, g);
-        s += vec_sumsq<VEC>(g, bad);
-        if constexpr (WRITE_ACC) st32<VEC>(acc + i, g);
-    }
+    if (K == 1) pass1_vectors<G, VEC, WRITE_ACC, 1>(gp, K, L, sa.inv_pre, inv_us, acc, s, bad);
+    else pass1_vectors<G, VEC, WRITE_ACC, 0>(gp, K, L, sa.inv_pre, inv_us, acc, s, bad);
     if (blockIdx.x == 0) {  // peeled head and ragged tail, one element per thread
         const unsigned long long extra = L.head + (L.n - L.tail0);
         for (unsigned long long j = threadIdx.x; j < extra; j += kThreads1) {
@@ -453,24 +484,15 @@ __device__ __forceinline__ void adam_vec(const float (&g)[VEC], const float (&ke
     }
 }
 
-template <class G, class W, int VEC, bool READ_ACC>
-__global__ void __launch_bounds__(kThreads3)
-adam_kernel(GradPtrs gp, int K, const float* __restrict__ acc, Layout L, AdamArgs a_arg,
-            float* __restrict__ master, float* __restrict__ m, float* __restrict__ v, uint16_t* __restrict__ w,
-            const unsigned long long* __restrict__ seg_end, const float* __restrict__ seg_wd, int nsegs,
-            const DevScalars* __restrict__ sc) {
-    // Programmatic dependent launch: everything below reads what pass 1 wrote.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (sc->overflow) return;  // skipped step: nothing is written
-    const float c = sc->coef;
-    AdamArgs a = a_arg;
-    const float inv_us = unscale_factor(a.post, sc->scale_used);
-    if (a.device_bc) {
-        a.lr = sc->lr;
-        a.step_size = sc->step_size;
-        a.bcs = sc->bc2_sqrt;
-    }
-
+// The vector loop of pass 2 (KFIX as in pass1_vectors).
+template <class G, class W, int VEC, bool READ_ACC, int KFIX>
+__device__ __forceinline__ void pass2_vectors(const GradPtrs& gp, int K_rt, const float* __restrict__ acc,
+                                              const Layout& L, const AdamArgs& a, float c, float inv_us,
+                                              float* __restrict__ master, float* __restrict__ m,
+                                              float* __restrict__ v, uint16_t* __restrict__ w,
+                                              const unsigned long long* __restrict__ seg_end,
+                                              const float* __restrict__ seg_wd, int nsegs) {
+    const int K = KFIX ? KFIX : K_rt;
     const unsigned long long stride = (unsigned long long)gridDim.x * kThreads3;
     unsigned long long v0 = (unsigned long long)blockIdx.x * kThreads3 + threadIdx.x;
     SegCursor cur{0, 0ull, 1.0f};
@@ -543,6 +565,30 @@ adam_kernel(GradPtrs gp, int K, const float* __restrict__ acc, Layout L, AdamArg
         st32<VEC>(v + i, vv);
         st16<W, VEC>(w + i, p);
     }
+}
+
+template <class G, class W, int VEC, bool READ_ACC>
+__global__ void __launch_bounds__(kThreads3)
+adam_kernel(GradPtrs gp, int K, const float* __restrict__ acc, Layout L, AdamArgs a_arg,
+            float* __restrict__ master, float* __restrict__ m, float* __restrict__ v, uint16_t* __restrict__ w,
+            const unsigned long long* __restrict__ seg_end, const float* __restrict__ seg_wd, int nsegs,
+            const DevScalars* __restrict__ sc) {
+    // Programmatic dependent launch: everything below reads what pass 1 wrote.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (sc->overflow) return;  // skipped step: nothing is written
+    const float c = sc->coef;
+    AdamArgs a = a_arg;
+    const float inv_us = unscale_factor(a.post, sc->scale_used);
+    if (a.device_bc) {
+        a.lr = sc->lr;
+        a.step_size = sc->step_size;
+        a.bcs = sc->bc2_sqrt;
+    }
+
+    if (K == 1)
+        pass2_vectors<G, W, VEC, READ_ACC, 1>(gp, K, acc, L, a, c, inv_us, master, m, v, w, seg_end, seg_wd, nsegs);
+    else
+        pass2_vectors<G, W, VEC, READ_ACC, 0>(gp, K, acc, L, a, c, inv_us, master, m, v, w, seg_end, seg_wd, nsegs);
     if (blockIdx.x == 0) {
         const unsigned long long extra = L.head + (L.n - L.tail0);
         for (unsigned long long j = threadIdx.x; j < extra; j += kThreads3) {
@@ -593,8 +639,7 @@ struct neox_shard {
     unsigned long long owned_bytes = 0;
     // profiling
     bool profiling = false;
-    bool mirror_stale = false;        // asynchronous steps ran since the last read
-    cudaStream_t last_stream = nullptr;
+    bool async_used = false;          // an asynchronous step was issued (replays may follow)
     cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};
     neox_profile prof{};
     std::string last_error;
@@ -773,19 +818,21 @@ void free_all(neox_shard* h) {
         if (e) cudaEventDestroy(e);
 }
 
-// Bring the host copy of the scaler state up to date after asynchronous steps.
+// Bring the host copy of the scaler state up to date.  Once asynchronous
+// steps were issued (possibly replayed from a CUDA graph, which this library
+// does not see), the device copy is the only current one: wait for the device
+// and read it.
 neox_status refresh_mirror(neox_shard* h) {
-    if (!h->mirror_stale) return NEOX_OK;
+    if (!h->async_used) return NEOX_OK;
     DeviceGuard g(h->device);
     cudaError_t e;
-    if ((e = cudaStreamSynchronize(h->last_stream)) != cudaSuccess) return cuda_fail(h, e, "waiting for asynchronous steps");
+    if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(h, e, "waiting for asynchronous steps");
     DevScalars r;
     if ((e = cudaMemcpy(&r, h->d_sc, sizeof(r), cudaMemcpyDeviceToHost)) != cudaSuccess)
         return cuda_fail(h, e, "reading the device scaler state");
     h->scale = r.scale;
     h->good = r.good;
     h->t = r.t;
-    h->mirror_stale = false;
     return NEOX_OK;
 }
 
@@ -793,8 +840,10 @@ neox_status refresh_mirror(neox_shard* h) {
 // device_bc = false: bias corrections from the host copy of t (synchronous
 // steps, whose caller keeps that copy current).  device_bc = true: the last
 // pass-1 block forms them from the device step count and writes `result`.
+// timed: record the profiling events around the two launches.
 neox_status enqueue_step(neox_shard* h, const void* const* grads, int32_t num_grads, void* params, float lr,
-                         const float* lr_dev, cudaStream_t st, bool device_bc, neox_step_result* result) {
+                         const float* lr_dev, cudaStream_t st, bool device_bc, neox_step_result* result,
+                         bool timed) {
     if (num_grads < 1 || num_grads > kMaxGrads) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "num_grads must be in [1, 64]");
     if (!grads) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "grads is NULL");
     if (!lr_dev && (!finite(lr) || lr < 0.0f)) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "lr must be finite and >= 0");
@@ -857,7 +906,6 @@ neox_status enqueue_step(neox_shard* h, const void* const* grads, int32_t num_gr
     a.inv_pre = sa.inv_pre;
     a.post = sa.post;
 
-    const bool timed = h->profiling && !device_bc;
     cudaError_t e;
     if (timed && (e = cudaEventRecord(h->ev[0], st)) != cudaSuccess) return cuda_fail(h, e, "cudaEventRecord");
     if (h->gdtype == NEOX_FP16) e = dispatch1v<F16>(h, vec, gp, num_grads, L, sa, acc, st);
@@ -1052,10 +1100,9 @@ neox_status neox_shard_set_state(neox_shard* h, float scale, int32_t good, int64
     if (!(scale > 0.0f) || !finite(scale) || good < 0 || t < 0)
         return fail(h, NEOX_ERR_INVALID_ARGUMENT, "state needs a finite scale > 0, good >= 0, t >= 0");
     DeviceGuard g(h->device);
-    if (h->mirror_stale) {
-        cudaError_t e0 = cudaStreamSynchronize(h->last_stream);
+    if (h->async_used) {
+        cudaError_t e0 = cudaDeviceSynchronize();
         if (e0 != cudaSuccess) return cuda_fail(h, e0, "waiting for asynchronous steps");
-        h->mirror_stale = false;
     }
     DevScalars s{};
     s.scale = scale;
@@ -1095,12 +1142,14 @@ neox_status neox_shard_step(neox_shard* h, const void* const* grads, int32_t num
     if (!h) return NEOX_ERR_INVALID_ARGUMENT;
     h->last_error.clear();
     if (!out) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "out is NULL");
-    if (neox_status s = refresh_mirror(h); s != NEOX_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
     DeviceGuard g(h->device);
     if (!g.ok) return fail(h, NEOX_ERR_CUDA, "cudaSetDevice failed");
-    const int64_t launches0 = h->prof.launches;
-    if (neox_status s = enqueue_step(h, grads, num_grads, params, lr, nullptr, st, false, nullptr); s != NEOX_OK)
+    // After asynchronous steps the host copy of t may be behind the device's:
+    // then the bias corrections are formed on the device as well.
+    if (neox_status s = enqueue_step(h, grads, num_grads, params, lr, nullptr, st, h->async_used, nullptr,
+                                     h->profiling);
+        s != NEOX_OK)
         return s;
     cudaError_t e;
     if ((e = cudaMemcpyAsync(h->h_sc, h->d_sc, sizeof(DevScalars), cudaMemcpyDeviceToHost, st)) != cudaSuccess)
@@ -1129,7 +1178,6 @@ neox_status neox_shard_step(neox_shard* h, const void* const* grads, int32_t num
         h->prof.last_grad_pass_ms = t01;
         h->prof.last_update_pass_ms = t12;
     }
-    (void)launches0;
     return NEOX_OK;
 }
 
@@ -1140,11 +1188,8 @@ neox_status neox_shard_step_async(neox_shard* h, const void* const* grads, int32
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
     DeviceGuard g(h->device);
     if (!g.ok) return fail(h, NEOX_ERR_CUDA, "cudaSetDevice failed");
-    if (neox_status s = enqueue_step(h, grads, num_grads, params, lr, lr_device, st, true, result); s != NEOX_OK)
-        return s;
-    h->mirror_stale = true;
-    h->last_stream = st;
-    return NEOX_OK;
+    h->async_used = true;
+    return enqueue_step(h, grads, num_grads, params, lr, lr_device, st, true, result, false);
 }
 
 }  // extern "C"

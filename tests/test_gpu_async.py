@@ -108,6 +108,8 @@ def test_async_step_in_cuda_graph():
         rb = _read_result(res_dev)
         ra = sa.step([g], a[3], lr)
         _same_result(ra, rb)
+        # replays run outside the library: its state read must still see them
+        assert sb.get_state() == (rb.loss_scale_next, rb.good_steps, rb.applied_steps)
     assert sb.get_state() == sa.get_state()
     _same_state(a, b)
     del graph

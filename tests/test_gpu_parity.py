@@ -296,3 +296,19 @@ def test_state_accounting_and_scratch():
     assert _abi.neox_model_state_bytes(175_000_000_000) == 2_800_000_000_000
     assert 0 < c.shard.scratch_bytes() < 1 << 20
     c.close()
+
+
+def test_huge_finite_gradients_are_not_overflow():
+    """FP16 gradients of about 1e4 carried at loss scale 2^-60 (floor 0): the
+    unscaled values (about 1e22) are finite although their squares pass FP32's
+    range.  No overflow, and the norm matches the oracle's double sum."""
+    n = 4099
+    c = ShardCase(n, hp=Hparams(clip_norm=1.0, init_scale=2.0 ** -60, min_scale=0.0, scale_window=1000),
+                  offsets={"all": 1}, lr=1e-3)
+    for s in range(1, 3):
+        synth.gpu_grad_normal16(c.g[0].t, 1e4, 1.0, c.seed, 0, s)
+        res, info = c.step()
+        assert info.overflow == 0 and res.overflow == 0 and info.norm > 1e22
+        c.check_result(res, info)
+        c.check_state()
+    c.close()
