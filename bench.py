@@ -46,6 +46,8 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["b200", "reference"], default="b200")
     p.add_argument("--workload", default="pythia_1p4b")
     p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--api", choices=["flat", "multi"], default="flat",
+                   help="flat: neox_shard_step; multi: neox_multi_step with one tensor per segment")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline")
     p.add_argument("--no-cpu-baseline", action="store_true")
     a = p.parse_args(argv)
@@ -222,8 +224,8 @@ def run_oracle_sample(wl, n_sample, steps, seconds, rank_seed=0):
             master[a:a + c] = 0
         elif init == "one":
             master[a:a + c] = 1
-    hp = oracle.OracleHparams(wl.beta1, wl.beta2, wl.eps, wl.clip, wl.predivide, wl.init_scale, 2.0, 1.0,
-                              wl.scale_window)
+    hp = oracle.OracleHparams(wl.beta1, wl.beta2, wl.eps, wl.clip, wl.predivide, wl.bench_scale or wl.init_scale,
+                              2.0, 1.0, wl.scale_window)
     sh = oracle.OracleShard(master, hp, wbf16=wl.bf16, gbf16=wl.bf16, segments=segs, default_wd=wl.weight_decay)
     grads = []
     for k in range(wl.K):
@@ -273,6 +275,14 @@ def run_reference(args):
 
 # ------------------------------------------------------------------ B200 arm
 
+def _at_offset(n, dtype, offset):
+    """A CUDA tensor of n elements starting `offset` elements past an
+    allocation boundary (the workload's misalignment)."""
+    import torch
+    base = torch.empty(n + offset, dtype=dtype, device="cuda")
+    return base.narrow(0, offset, n)
+
+
 def build_gpu_workload(wl, rank):
     import torch
 
@@ -281,29 +291,77 @@ def build_gpu_workload(wl, rank):
     n = wl.numel
     dt = torch.bfloat16 if wl.bf16 else torch.float16
     seed = wl.seed + 1000 * rank
-    master = torch.empty(n, dtype=torch.float32, device="cuda")
+    off = wl.elem_offset
+    scale = wl.bench_scale or wl.init_scale
+    master = _at_offset(n, torch.float32, off)
     synth.gpu_master_normal(master, wl.master_sigma, seed)
     for off, cnt, _, init in (wl.segments or []):
         if init == "zero":
             master[off:off + cnt].zero_()
         elif init == "one":
             master[off:off + cnt].fill_(1.0)
-    m = torch.zeros_like(master)
-    v = torch.zeros_like(master)
-    params = master.to(dt)
+    m = _at_offset(n, torch.float32, off).zero_()
+    v = _at_offset(n, torch.float32, off).zero_()
+    params = _at_offset(n, dt, off)
+    params.copy_(master.to(dt))
     grads = []
     for k in range(wl.K):
-        g = torch.empty(n, dtype=dt, device="cuda")
+        g = _at_offset(n, dt, off)
         if wl.grad_dist == "t3":
-            synth.gpu_grad_t3_16(g, wl.init_scale, seed, k, 1, wl.bf16)
+            synth.gpu_grad_t3_16(g, scale, seed, k, 1, wl.bf16)
         else:
-            synth.gpu_grad_normal16(g, wl.grad_sigma, wl.init_scale, seed, k, 1, wl.bf16)
+            synth.gpu_grad_normal16(g, wl.grad_sigma, scale, seed, k, 1, wl.bf16)
         grads.append(g)
-    hp = Hparams(wl.beta1, wl.beta2, wl.eps, wl.clip, wl.predivide, wl.init_scale, 2.0, 1.0, wl.scale_window)
+    hp = Hparams(wl.beta1, wl.beta2, wl.eps, wl.clip, wl.predivide, scale, 2.0, 1.0, wl.scale_window)
     shard = NeoxShard(master, m, v, hp, wdtype=dt, gdtype=dt, segments=wl.seg_table(),
                       weight_decay=wl.weight_decay, max_grads=wl.K)
     torch.cuda.synchronize()
     return shard, grads, params, (master, m, v)
+
+
+def run_multi(args):
+    """The multi-tensor step on the same workload: one tensor per segment, as
+    views of the same device buffers, timed like the flat step."""
+    import torch
+
+    from mixed_precision_zero_b200 import Hparams, NeoxMultiShard
+    from synth import workloads as W
+    torch.cuda.set_device(0)
+    wl = W.ALL[args.workload]()
+    shard, grads, params, (master, m, v) = build_gpu_workload(wl, 0)
+    shard.close()
+    segs = wl.seg_table() or [(0, wl.numel, wl.weight_decay)]
+    scale = wl.bench_scale or wl.init_scale
+    hp = Hparams(wl.beta1, wl.beta2, wl.eps, wl.clip, wl.predivide, scale, 2.0, 1.0, wl.scale_window)
+    multi = NeoxMultiShard([{"master": master[o:o + c], "exp_avg": m[o:o + c], "exp_avg_sq": v[o:o + c],
+                             "params": params[o:o + c], "grads": [g[o:o + c] for g in grads], "weight_decay": w}
+                            for o, c, w in segs], hp)
+    for _ in range(args.warmup):
+        multi.step(wl.lr)
+    t0 = multi.get_state()[2]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with ClockSampler(0) as clocks:
+        e0.record()
+        for _ in range(args.steps):
+            multi.step(wl.lr)
+        e1.record()
+        torch.cuda.synchronize()
+    assert multi.get_state()[2] - t0 == args.steps
+    ms = e0.elapsed_time(e1)
+    p1b, p2b = alg_bytes_per_param(wl.K, False)
+    peak, kind = hbm_peak()
+    line = {"metric": METRIC, "value": wl.numel * args.steps / (ms * 1e-3) / 1e9, "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "impl": "b200",
+            "config": {"workload": wl.name, "api": "neox_multi_step", "tensors": len(segs)},
+            "hbm": {"step_gbs": (p1b + p2b) * wl.numel / (ms / args.steps * 1e-3) / 1e9,
+                    "step_frac": (p1b + p2b) * wl.numel / (ms / args.steps * 1e-3) / 1e9 / peak, "peak_gbs": peak,
+                    "peak_kind": kind},
+            "clocks": clocks.summary()}
+    multi.close()
+    print(json.dumps(line), flush=True)
+    return 0
 
 
 def run_b200(args):
@@ -429,6 +487,7 @@ def run_b200(args):
         "dtype": "f32", "data": "synthetic",
         "config": {"workload": wl.name, "numel_per_rank": wl.numel, "segments": len(wl.segments or [1]),
                    "grad_buffers": wl.K, "weights": "bf16" if wl.bf16 else "fp16",
+                   "element_offset": wl.elem_offset, "loss_scale": wl.bench_scale or wl.init_scale,
                    "state": "fp32 master/m/v",
                    "l2": f"inputs {(14 + 2 * wl.K) * wl.numel / 1e9:.1f} GB per rank >> 126 MB L2; no flush",
                    "parallelism": f"{ws} independent shard(s), one per GPU"},
@@ -460,6 +519,8 @@ def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.api == "multi":
+        return run_multi(args)
     return run_b200(args)
 
 

@@ -132,9 +132,10 @@ neox_status neox_shard_create(const neox_shard_desc* desc, const neox_hparams* h
  *   lr:        learning rate of this step, finite and >= 0;
  *   out:       host result, filled on NEOX_OK.
  * Arrays may start at any element offset: when every array has the same
- * address residue (mod 16 bytes, in elements) the kernels peel a short head
- * and use 16-byte vectors, otherwise they fall back to narrower vectors, with
- * the same results.  The call is stream-ordered and returns after the step
+ * element offset from a 128-byte line the kernels peel a head of up to 63
+ * elements and stream whole lines with 16-byte vectors; with only a common
+ * 16-byte residue they peel less; otherwise they fall back to narrower
+ * vectors.  The results are the same in every case.  The call is stream-ordered and returns after the step
  * has finished on the GPU (it synchronises cuda_stream only).  Overflow is
  * not an error: it returns NEOX_OK with out->overflow = 1.  On
  * NEOX_ERR_INVALID_ARGUMENT nothing was launched; on NEOX_ERR_CUDA the shard
@@ -208,6 +209,64 @@ typedef struct {
 neox_status neox_shard_set_profiling(neox_shard* h, int32_t enable);
 neox_status neox_shard_get_profile(const neox_shard* h, neox_profile* out);
 neox_status neox_shard_reset_profile(neox_shard* h);
+
+/* ------------------------------------------------------------------------
+ * Multi-tensor (non-flat) shard.
+ *
+ * The same step over a shard made of many separately allocated tensors (one
+ * shard per parameter, as FSDP does when it shards parameter by parameter
+ * instead of flattening them): mathematically the flat step over the
+ * tensors' concatenation with one weight-decay segment per tensor, including
+ * the single global norm, flag and scaler.  "OPT: Open Pre-trained
+ * Transformer Language Models" (ai-papers.xuzou.cn summary), sections
+ * "计算设置" / "方法适配": FSDP shards the model state across ranks.
+ *
+ * All pointers are bound at create: every tensor's FP32 master / exp_avg /
+ * exp_avg_sq (4-byte aligned), its 16-bit working weights (params) and its
+ * num_grads 16-bit gradient buffers (2-byte aligned), all device memory the
+ * caller owns and keeps alive.  Each tensor chooses its own vector width and
+ * head peel from its own pointers.  A tensor may have numel 0 (its pointers
+ * are then ignored).  The steps are then launched with only the learning
+ * rate; both kernels walk a chunk table (up to 65,536 elements per chunk).
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    uint64_t numel;
+    float weight_decay;
+    float* master;
+    float* exp_avg;
+    float* exp_avg_sq;
+    void* params;                 /* 16-bit working weights                   */
+    const void* const* grads;     /* host array of num_grads device pointers  */
+} neox_tensor;
+
+typedef struct {
+    int32_t ntensors;             /* >= 0                                     */
+    int32_t num_grads;            /* K in [1, 64], the same for every tensor  */
+    neox_dtype wdtype, gdtype;
+    const neox_tensor* tensors;   /* host array of ntensors                   */
+} neox_tensor_set;
+
+typedef struct neox_multi neox_multi;
+
+/* Validate every tensor (NEOX_ERR_INVALID_ARGUMENT before any CUDA call),
+ * build the chunk table and copy it, the tensor table and the gradient
+ * pointer table to the device. */
+neox_status neox_multi_create(const neox_tensor_set* set, const neox_hparams* hp, int device, neox_multi** out);
+/* One step, as neox_shard_step (blocking on cuda_stream). */
+neox_status neox_multi_step(neox_multi* h, float lr, void* cuda_stream, neox_step_result* out);
+/* One step, as neox_shard_step_async (no host read-back, graph-capturable). */
+neox_status neox_multi_step_async(neox_multi* h, float lr, const float* lr_device, void* cuda_stream,
+                                  neox_step_result* result);
+/* Point the tensors at other gradient buffers: `grads` is a host array of
+ * ntensors * num_grads device pointers (tensor-major), each with the same
+ * address residue as the buffer it replaces (the tensor's vector layout is
+ * kept).  Waits for the device, then copies the table (synchronous). */
+neox_status neox_multi_rebind_grads(neox_multi* h, const void* const* grads);
+neox_status neox_multi_set_hparams(neox_multi* h, const neox_hparams* hp);
+neox_status neox_multi_get_state(const neox_multi* h, float* scale, int32_t* good, int64_t* t);
+neox_status neox_multi_set_state(neox_multi* h, float scale, int32_t good, int64_t t);
+void neox_multi_destroy(neox_multi* h);
+const char* neox_multi_last_error(const neox_multi* h);
 
 /* ------------------------------------------------------------------------
  * Step without a handle and without any allocation.

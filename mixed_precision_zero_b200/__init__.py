@@ -21,9 +21,12 @@ from ._abi import (NEOX_BF16, NEOX_ERR_CUDA, NEOX_ERR_INVALID_ARGUMENT, NEOX_ERR
                    neox_shard_create, neox_shard_desc, neox_shard_destroy, neox_shard_get_profile,
                    neox_shard_get_state, neox_shard_reset_profile, neox_shard_scratch_bytes,
                    neox_shard_set_hparams, neox_shard_set_profiling, neox_shard_set_state,
-                   neox_shard_step, neox_shard_step_async, neox_status_string, neox_step_result)
+                   neox_shard_step, neox_shard_step_async, neox_status_string, neox_step_result,
+                   neox_tensor, neox_tensor_set, neox_multi_create, neox_multi_step, neox_multi_step_async,
+                   neox_multi_rebind_grads, neox_multi_get_state, neox_multi_set_state,
+                   neox_multi_set_hparams, neox_multi_destroy)
 
-__all__ = ["NeoxShard", "Hparams", "NeoxError", "neox_shard_create", "neox_shard_step",
+__all__ = ["NeoxShard", "NeoxMultiShard", "Hparams", "NeoxError", "neox_shard_create", "neox_shard_step",
            "neox_shard_destroy", "neox_shard_set_hparams", "neox_shard_get_state",
            "neox_shard_set_state", "neox_status_string", "neox_last_error", "neox_model_state_bytes"]
 
@@ -137,6 +140,84 @@ class NeoxShard:
     def close(self) -> None:
         if getattr(self, "handle", None):
             neox_shard_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class NeoxMultiShard:
+    """A shard made of separately allocated tensors (one per parameter), stepped
+    as one: `tensors` is a list of dicts with keys master, exp_avg, exp_avg_sq
+    (float32 CUDA tensors), params (16-bit), grads (list of K 16-bit tensors)
+    and weight_decay.  All buffers are bound here and must stay alive."""
+
+    def __init__(self, tensors, hp: Hparams | None = None, *, device: int | None = None):
+        import torch
+        hp = hp or Hparams()
+        K = len(tensors[0]["grads"]) if tensors else 1
+        self._keep = tensors
+        self._grad_arrays = []
+        descs = []
+        wd_t = gd_t = None
+        for t in tensors:
+            n = t["master"].numel()
+            for x in (t["master"], t["exp_avg"], t["exp_avg_sq"]):
+                if x.dtype != torch.float32 or x.numel() != n or not x.is_contiguous():
+                    raise ValueError("master/exp_avg/exp_avg_sq must be contiguous float32 tensors of equal length")
+            if len(t["grads"]) != K:
+                raise ValueError("every tensor needs the same number of gradient buffers")
+            for g in [t["params"], *t["grads"]]:
+                if g.numel() != n or not g.is_contiguous():
+                    raise ValueError("params/grads must be contiguous and as long as master")
+            wd_t = wd_t or t["params"].dtype
+            gd_t = gd_t or t["grads"][0].dtype
+            garr = (ctypes.c_void_p * K)(*[g.data_ptr() for g in t["grads"]])
+            self._grad_arrays.append(garr)
+            descs.append(neox_tensor(n, float(t.get("weight_decay", 0.0)), t["master"].data_ptr(),
+                                     t["exp_avg"].data_ptr(), t["exp_avg_sq"].data_ptr(), t["params"].data_ptr(),
+                                     ctypes.cast(garr, ctypes.POINTER(ctypes.c_void_p))))
+        self._descs = (neox_tensor * max(1, len(descs)))(*descs)
+        wcode = NEOX_BF16 if wd_t == torch.bfloat16 else NEOX_FP16
+        gcode = NEOX_BF16 if gd_t == torch.bfloat16 else NEOX_FP16
+        tset = neox_tensor_set(len(descs), K, wcode, gcode, ctypes.cast(self._descs, ctypes.POINTER(neox_tensor)))
+        self.device = torch.cuda.current_device() if device is None else device
+        self.handle = neox_multi_create(tset, hp.c(), self.device)
+
+    @staticmethod
+    def _sp(stream, device):
+        import torch
+        if stream is None:
+            stream = torch.cuda.current_stream(device)
+        return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+    def step(self, lr: float, stream=None) -> neox_step_result:
+        return neox_multi_step(self.handle, lr, self._sp(stream, self.device))
+
+    def step_async(self, lr: float = 0.0, *, result=None, lr_device=None, stream=None) -> None:
+        neox_multi_step_async(self.handle, lr, self._sp(stream, self.device),
+                              None if result is None else result.data_ptr(),
+                              None if lr_device is None else lr_device.data_ptr())
+
+    def rebind_grads(self, grads_per_tensor) -> None:
+        ptrs = [g.data_ptr() for gs in grads_per_tensor for g in gs]
+        neox_multi_rebind_grads(self.handle, ptrs)
+
+    def get_state(self):
+        return neox_multi_get_state(self.handle)
+
+    def set_state(self, scale: float, good: int, t: int) -> None:
+        neox_multi_set_state(self.handle, scale, good, t)
+
+    def set_hparams(self, hp: Hparams) -> None:
+        neox_multi_set_hparams(self.handle, hp.c())
+
+    def close(self) -> None:
+        if getattr(self, "handle", None):
+            neox_multi_destroy(self.handle)
             self.handle = None
 
     def __del__(self):

@@ -53,6 +53,17 @@ class neox_scaler_state(ctypes.Structure):
     _fields_ = [("scale", ctypes.c_float), ("good", ctypes.c_int32), ("t", ctypes.c_int64)]
 
 
+class neox_tensor(ctypes.Structure):
+    _fields_ = [("numel", ctypes.c_uint64), ("weight_decay", ctypes.c_float),
+                ("master", ctypes.c_void_p), ("exp_avg", ctypes.c_void_p), ("exp_avg_sq", ctypes.c_void_p),
+                ("params", ctypes.c_void_p), ("grads", ctypes.POINTER(ctypes.c_void_p))]
+
+
+class neox_tensor_set(ctypes.Structure):
+    _fields_ = [("ntensors", ctypes.c_int32), ("num_grads", ctypes.c_int32), ("wdtype", ctypes.c_int),
+                ("gdtype", ctypes.c_int), ("tensors", ctypes.POINTER(neox_tensor))]
+
+
 class neox_profile(ctypes.Structure):
     _fields_ = [("steps", ctypes.c_int64), ("launches", ctypes.c_int64),
                 ("grad_pass_ms", ctypes.c_double), ("update_pass_ms", ctypes.c_double),
@@ -109,6 +120,26 @@ def lib() -> ctypes.CDLL:
                                               ctypes.c_int32, ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p,
                                               ctypes.POINTER(neox_step_result)]
         L.neox_shard_step_noalloc.restype = S
+        L.neox_multi_create.argtypes = [ctypes.POINTER(neox_tensor_set), ctypes.POINTER(neox_hparams), ctypes.c_int,
+                                        ctypes.POINTER(_H)]
+        L.neox_multi_create.restype = S
+        L.neox_multi_step.argtypes = [_H, ctypes.c_float, ctypes.c_void_p, ctypes.POINTER(neox_step_result)]
+        L.neox_multi_step.restype = S
+        L.neox_multi_step_async.argtypes = [_H, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+        L.neox_multi_step_async.restype = S
+        L.neox_multi_rebind_grads.argtypes = [_H, ctypes.POINTER(ctypes.c_void_p)]
+        L.neox_multi_rebind_grads.restype = S
+        L.neox_multi_set_hparams.argtypes = [_H, ctypes.POINTER(neox_hparams)]
+        L.neox_multi_set_hparams.restype = S
+        L.neox_multi_get_state.argtypes = [_H, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int32),
+                                           ctypes.POINTER(ctypes.c_int64)]
+        L.neox_multi_get_state.restype = S
+        L.neox_multi_set_state.argtypes = [_H, ctypes.c_float, ctypes.c_int32, ctypes.c_int64]
+        L.neox_multi_set_state.restype = S
+        L.neox_multi_destroy.argtypes = [_H]
+        L.neox_multi_destroy.restype = None
+        L.neox_multi_last_error.argtypes = [_H]
+        L.neox_multi_last_error.restype = ctypes.c_char_p
         L.neox_noalloc_last_error.argtypes = []
         L.neox_noalloc_last_error.restype = ctypes.c_char_p
         _lib = L
@@ -212,3 +243,62 @@ def neox_shard_step_noalloc(desc: neox_shard_desc, hp: neox_hparams, state: neox
     if st != NEOX_OK:
         raise NeoxError(st, lib().neox_noalloc_last_error().decode())
     return res
+
+
+# ---- multi-tensor shard -----------------------------------------------------------
+
+def _merr(h):
+    return lib().neox_multi_last_error(h).decode()
+
+
+def neox_multi_create(tset: neox_tensor_set, hp: neox_hparams, device: int) -> int:
+    h = _H()
+    st = lib().neox_multi_create(ctypes.byref(tset), ctypes.byref(hp), device, ctypes.byref(h))
+    if st != NEOX_OK:
+        raise NeoxError(st, _merr(None))
+    return h.value
+
+
+def neox_multi_step(h: int, lr: float, stream: int) -> neox_step_result:
+    res = neox_step_result()
+    st = lib().neox_multi_step(h, lr, stream, ctypes.byref(res))
+    if st != NEOX_OK:
+        raise NeoxError(st, _merr(h))
+    return res
+
+
+def neox_multi_step_async(h: int, lr: float, stream: int, result_ptr=None, lr_device_ptr=None) -> None:
+    st = lib().neox_multi_step_async(h, lr, lr_device_ptr, stream, result_ptr)
+    if st != NEOX_OK:
+        raise NeoxError(st, _merr(h))
+
+
+def neox_multi_rebind_grads(h: int, grad_ptrs) -> None:
+    arr = (ctypes.c_void_p * len(grad_ptrs))(*grad_ptrs)
+    st = lib().neox_multi_rebind_grads(h, arr)
+    if st != NEOX_OK:
+        raise NeoxError(st, _merr(h))
+
+
+def neox_multi_get_state(h: int):
+    s, g, t = ctypes.c_float(), ctypes.c_int32(), ctypes.c_int64()
+    st = lib().neox_multi_get_state(h, ctypes.byref(s), ctypes.byref(g), ctypes.byref(t))
+    if st != NEOX_OK:
+        raise NeoxError(st, _merr(h))
+    return s.value, g.value, t.value
+
+
+def neox_multi_set_state(h: int, scale: float, good: int, t: int) -> None:
+    st = lib().neox_multi_set_state(h, scale, good, t)
+    if st != NEOX_OK:
+        raise NeoxError(st, _merr(h))
+
+
+def neox_multi_set_hparams(h: int, hp: neox_hparams) -> None:
+    st = lib().neox_multi_set_hparams(h, ctypes.byref(hp))
+    if st != NEOX_OK:
+        raise NeoxError(st, _merr(h))
+
+
+def neox_multi_destroy(h: int) -> None:
+    lib().neox_multi_destroy(h)

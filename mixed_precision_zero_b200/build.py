@@ -21,7 +21,7 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-shared",
                      "-Xptxas", "-v", "-I", INCLUDE]
 
-SOURCES = [os.path.join(PKG, "csrc", "neox_shard.cu")]
+SOURCES = [os.path.join(PKG, "csrc", "neox_shard.cu"), os.path.join(PKG, "csrc", "neox_multi.cu")]
 LIB = os.path.join(PKG, "libneoxshard.so")
 
 
@@ -33,7 +33,7 @@ def _stale(target: str, deps) -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    deps = SOURCES + [os.path.join(INCLUDE, "neox_shard.h")]
+    deps = SOURCES + [os.path.join(INCLUDE, "neox_shard.h"), os.path.join(PKG, "csrc", "neox_common.cuh")]
     if force or _stale(LIB, deps):
         tmp = LIB + f".tmp{os.getpid()}"
         cmd = [NVCC, *NVCC_FLAGS, "-o", tmp, *SOURCES]

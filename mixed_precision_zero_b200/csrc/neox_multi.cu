@@ -1,0 +1,622 @@
+// neox_multi.cu -- the per-rank mixed-precision optimizer step over a shard
+// made of many separately allocated tensors (per-parameter sharding, as in
+// FSDP with one shard per parameter), in one pair of launches.
+//
+// The step is the flat step of neox_shard.cu over the concatenation of the
+// tensors, each tensor being one weight-decay segment: the same ingest,
+// overflow flag, global norm, loss scaler, clip coefficient, AdamW and cast,
+// with the same per-element arithmetic (neox_common.cuh).  Pages followed:
+// "OPT: Open Pre-trained Transformer Language Models" (ai-papers.xuzou.cn
+// summary), "方法适配" (method adaptation) and "计算设置" (compute setup): FSDP
+// shards model state across ranks, Adam state FP32, weights FP16, dynamic
+// loss scaling, gradient pre-divide and clipping.
+//
+// Work decomposition: both kernels walk the tensors in order and cover each
+// tensor grid-stride across the whole grid, exactly as the flat kernels cover
+// the flat shard (an outer loop over tensors; no synchronisation between
+// tensors).  Each tensor keeps its own vector width and peeled head, chosen
+// from its own pointers; its head and ragged tail are done by block
+// (tensor index mod grid).  A per-block chunk decomposition was measured 11%
+// slower: every block then streams its own distant region instead of all
+// warps streaming one window together.
+
+#include "neox_shard.h"
+#include "neox_common.cuh"
+
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+namespace {
+
+constexpr int kMtThreads1 = 512;
+constexpr int kMtThreads3 = 256;
+constexpr int kMtDescBatch = 256;  // pass 1: tensor descriptors staged in shared memory at a time
+constexpr int kMtDescBatch3 = 768; // pass 2: 60 KB of descriptors (dynamic shared memory)
+
+struct alignas(16) MtTensor {
+    float* master;
+    float* m;
+    float* v;
+    uint16_t* w;
+    unsigned long long numel, head, nvec, tail0;
+    float wd;
+    int vec;
+    int gbase;  // the tensor's K gradient pointers are gtab[gbase .. gbase + K)
+    int pad_;
+};
+
+static_assert(sizeof(MtTensor) % 16 == 0, "descriptors are copied as 16-byte words");
+
+// Copy descriptors [base, base + cnt) into shared memory (all threads).  A
+// warp then reads each tensor's pointers from shared memory instead of
+// waiting on a dependent global load at every tensor boundary.
+__device__ __forceinline__ void stage_descriptors(const MtTensor* __restrict__ tens, int base, int cnt,
+                                                  MtTensor* tsh) {
+    constexpr int W = sizeof(MtTensor) / 16;
+    const int4* src = reinterpret_cast<const int4*>(tens + base);
+    int4* dst = reinterpret_cast<int4*>(tsh);
+    __syncthreads();  // the previous batch is no longer read
+    for (int i = threadIdx.x; i < cnt * W; i += blockDim.x) dst[i] = __ldg(src + i);
+    __syncthreads();
+}
+
+// ---------------------------------------------------------------- pass 1
+template <class G, int VEC, int KFIX>
+__device__ __forceinline__ void mt_p1_tensor(const GradTab& gp, int K_rt, const MtTensor& T, float inv_pre,
+                                             float inv_us, double& s, int& bad) {
+    const int K = KFIX ? KFIX : K_rt;
+    constexpr int U = KFIX ? 4 : 2;
+    const unsigned long long stride = (unsigned long long)gridDim.x * kMtThreads1;
+    unsigned long long v = (unsigned long long)blockIdx.x * kMtThreads1 + threadIdx.x;
+    for (; v + (U - 1) * stride < T.nvec; v += U * stride) {
+        float g[U][VEC];
+        ingest_batch<G, VEC, U>(gp, K, T.head + v * VEC, stride * VEC, inv_pre, inv_us, g);
+#pragma unroll
+        for (int u = 0; u < U; u++) s += vec_sumsq<VEC>(g[u], bad);
+    }
+    // The last (fewer than U) strides: still U loads in flight.  Most tensors
+    // of a model are shorter than U grid strides, so this batch does most of
+    // their work.  The thread's vectors are summed in the same order.
+    if (v < T.nvec) {
+        bool ok[U];
+#pragma unroll
+        for (int u = 0; u < U; u++) ok[u] = v + u * stride < T.nvec;
+        float g[U][VEC];
+        ingest_batch_pred<G, VEC, U>(gp, K, T.head + v * VEC, stride * VEC, ok, inv_pre, inv_us, g);
+#pragma unroll
+        for (int u = 0; u < U; u++)
+            if (ok[u]) s += vec_sumsq<VEC>(g[u], bad);
+    }
+}
+
+template <class G, int KFIX>
+__device__ __forceinline__ void mt_p1_dispatch(const MtTensor& T, const GradTab& gp, int K, float inv_pre,
+                                               float inv_us, double& s, int& bad) {
+    switch (T.vec) {
+        case 8: mt_p1_tensor<G, 8, KFIX>(gp, K, T, inv_pre, inv_us, s, bad); break;
+        case 4: mt_p1_tensor<G, 4, KFIX>(gp, K, T, inv_pre, inv_us, s, bad); break;
+        case 2: mt_p1_tensor<G, 2, KFIX>(gp, K, T, inv_pre, inv_us, s, bad); break;
+        default: mt_p1_tensor<G, 1, KFIX>(gp, K, T, inv_pre, inv_us, s, bad); break;
+    }
+}
+
+template <class G>
+__global__ void __launch_bounds__(kMtThreads1, 1024 / kMtThreads1)
+mt_stats_kernel(const MtTensor* __restrict__ tens, int ntensors, const uint16_t* const* __restrict__ gtab, int K,
+                ScalerArgs sa, double* __restrict__ part_s, int* __restrict__ part_b, DevScalars* __restrict__ sc) {
+    __shared__ double sh_s[kMtThreads1 / 32];
+    __shared__ int sh_b[kMtThreads1 / 32];
+    __shared__ bool is_last;
+    __shared__ MtTensor tsh[kMtDescBatch];
+    const float inv_us = unscale_factor(sa.post, sc->scale);
+    double s = 0.0;
+    int bad = 0;
+    for (int base = 0; base < ntensors; base += kMtDescBatch) {
+    const int cnt = ntensors - base < kMtDescBatch ? ntensors - base : kMtDescBatch;
+    stage_descriptors(tens, base, cnt, tsh);
+    for (int ti = base; ti < base + cnt; ti++) {
+        const MtTensor T = tsh[ti - base];  // by value: registers, not re-read after stores
+        if (T.numel == 0) continue;
+        const GradTab gp{gtab, T.gbase};
+        if (K == 1) mt_p1_dispatch<G, 1>(T, gp, K, sa.inv_pre, inv_us, s, bad);
+        else mt_p1_dispatch<G, 0>(T, gp, K, sa.inv_pre, inv_us, s, bad);
+        if ((unsigned)ti % gridDim.x == blockIdx.x) {  // this tensor's head and tail
+            const unsigned long long extra = T.head + (T.numel - T.tail0);
+            for (unsigned long long j = threadIdx.x; j < extra; j += kMtThreads1) {
+                const unsigned long long i = j < T.head ? j : T.tail0 + (j - T.head);
+                float g[1];
+                ingest<G, 1>(gp, K, i, sa.inv_pre, inv_us, g);
+                s += vec_sumsq<1>(g, bad);
+            }
+        }
+    }
+    }
+    finish_pass1<kMtThreads1>(s, bad, part_s, part_b, sc, sa, sh_s, sh_b, &is_last);
+}
+
+// ---------------------------------------------------------------- pass 2
+template <class G, class W, int VEC, int KFIX>
+__device__ __forceinline__ void mt_p2_tensor(const GradTab& gp, int K_rt, const MtTensor& T, float keep1, float c,
+                                             float inv_us, const AdamArgs& a) {
+    const int K = KFIX ? KFIX : K_rt;
+    float keep[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; e++) keep[e] = keep1;
+    const unsigned long long stride = (unsigned long long)gridDim.x * kMtThreads3;
+    float* __restrict__ master = T.master;
+    float* __restrict__ m = T.m;
+    float* __restrict__ v = T.v;
+    uint16_t* __restrict__ w = T.w;
+    const unsigned long long nvec = T.nvec, head = T.head;
+    for (unsigned long long vi = (unsigned long long)blockIdx.x * kMtThreads3 + threadIdx.x; vi < nvec; vi += stride) {
+        const unsigned long long i = head + vi * VEC;
+        float g[VEC], p[VEC], mm[VEC], vv[VEC];
+        ingest<G, VEC>(gp, K, i, a.inv_pre, inv_us, g);
+        ld32<VEC>(master + i, p);
+        ld32<VEC>(m + i, mm);
+        ld32<VEC>(v + i, vv);
+        adam_vec<VEC>(g, keep, c, a, p, mm, vv);
+        st32<VEC>(master + i, p);
+        st32<VEC>(m + i, mm);
+        st32<VEC>(v + i, vv);
+        st16<W, VEC>(w + i, p);
+    }
+}
+
+template <class G, class W, int KFIX>
+__device__ __forceinline__ void mt_p2_dispatch(const MtTensor& T, const GradTab& gp, int K, float keep1, float c,
+                                               float inv_us, const AdamArgs& a) {
+    switch (T.vec) {
+        case 8: mt_p2_tensor<G, W, 8, KFIX>(gp, K, T, keep1, c, inv_us, a); break;
+        case 4: mt_p2_tensor<G, W, 4, KFIX>(gp, K, T, keep1, c, inv_us, a); break;
+        case 2: mt_p2_tensor<G, W, 2, KFIX>(gp, K, T, keep1, c, inv_us, a); break;
+        default: mt_p2_tensor<G, W, 1, KFIX>(gp, K, T, keep1, c, inv_us, a); break;
+    }
+}
+
+template <class G, class W>
+__global__ void __launch_bounds__(kMtThreads3)
+mt_adam_kernel(const MtTensor* __restrict__ tens, int ntensors, const uint16_t* const* __restrict__ gtab, int K,
+               AdamArgs a_arg, const DevScalars* __restrict__ sc) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // pass 1's results
+    if (sc->overflow) return;
+    const float c = sc->coef;
+    AdamArgs a = a_arg;
+    const float inv_us = unscale_factor(a.post, sc->scale_used);
+    if (a.device_bc) {
+        a.lr = sc->lr;
+        a.step_size = sc->step_size;
+        a.bcs = sc->bc2_sqrt;
+    }
+    // Descriptors are staged in the dynamic shared memory, whose size (set at
+    // launch) also holds the kernel to 3 blocks per SM: a measured 4% better
+    // for this read/write stream than the 4 blocks its registers would allow.
+    extern __shared__ MtTensor tsh_dyn[];
+    for (int base = 0; base < ntensors; base += kMtDescBatch3) {
+    const int cnt = ntensors - base < kMtDescBatch3 ? ntensors - base : kMtDescBatch3;
+    stage_descriptors(tens, base, cnt, tsh_dyn);
+    for (int ti = base; ti < base + cnt; ti++) {
+        const MtTensor T = tsh_dyn[ti - base];  // by value: registers, not re-read after stores
+        if (T.numel == 0) continue;
+        const GradTab gp{gtab, T.gbase};
+        const float keep1 = __fsub_rn(1.0f, __fmul_rn(a.lr, T.wd));  // fl32(1 - fl32(lr * wd))
+        if (K == 1) mt_p2_dispatch<G, W, 1>(T, gp, K, keep1, c, inv_us, a);
+        else mt_p2_dispatch<G, W, 0>(T, gp, K, keep1, c, inv_us, a);
+        if ((unsigned)ti % gridDim.x == blockIdx.x) {  // this tensor's head and tail
+            const unsigned long long extra = T.head + (T.numel - T.tail0);
+            for (unsigned long long j = threadIdx.x; j < extra; j += kMtThreads3) {
+                const unsigned long long i = j < T.head ? j : T.tail0 + (j - T.head);
+                float g[1], p[1] = {T.master[i]}, mm[1] = {T.m[i]}, vv[1] = {T.v[i]}, keep[1] = {keep1};
+                ingest<G, 1>(gp, K, i, a.inv_pre, inv_us, g);
+                adam_vec<1>(g, keep, c, a, p, mm, vv);
+                T.master[i] = p[0];
+                T.m[i] = mm[0];
+                T.v[i] = vv[0];
+                T.w[i] = W::enc(p[0]);
+            }
+        }
+    }
+    }
+}
+
+}  // namespace
+
+// ====================================================================== host
+
+struct neox_multi {
+    int device = 0;
+    int sm_count = 0;
+    int ntensors = 0;
+    int K = 1;
+    neox_dtype wdtype = NEOX_FP16, gdtype = NEOX_FP16;
+    neox_hparams hp{};
+    unsigned long long numel = 0;
+    unsigned long long max_vecs = 0;  // vectors of the largest tensor
+    int grid2 = 1;                    // pass-2 grid (resident blocks, set at create)
+    float scale = 1.0f;
+    int32_t good = 0;
+    long long t = 0;
+    bool async_used = false;
+    int max_parts = 0;
+    MtTensor* d_tens = nullptr;
+    const uint16_t** d_gtab = nullptr;
+    DevScalars* d_sc = nullptr;
+    double* d_part_s = nullptr;
+    int* d_part_b = nullptr;
+    DevScalars* h_sc = nullptr;
+    std::vector<MtTensor> tens;  // host copy (pointers and layouts)
+    std::string last_error;
+};
+
+namespace {
+
+thread_local std::string g_multi_create_error;
+
+neox_status mfail(neox_multi* h, neox_status st, const std::string& msg) {
+    if (h) h->last_error = msg; else g_multi_create_error = msg;
+    return st;
+}
+
+neox_status mcuda_fail(neox_multi* h, cudaError_t e, const char* what) {
+    return mfail(h, e == cudaErrorMemoryAllocation ? NEOX_ERR_OUT_OF_MEMORY : NEOX_ERR_CUDA,
+                 std::string(what) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")");
+}
+
+void mfree(neox_multi* h) {
+    if (h->d_tens) cudaFree(h->d_tens);
+    if (h->d_gtab) cudaFree(h->d_gtab);
+    if (h->d_sc) cudaFree(h->d_sc);
+    if (h->d_part_s) cudaFree(h->d_part_s);
+    if (h->d_part_b) cudaFree(h->d_part_b);
+    if (h->h_sc) cudaFreeHost(h->h_sc);
+}
+
+// Pointer table and layout of every tensor; returns an error message or "".
+std::string build_tables(const neox_tensor_set* set, std::vector<MtTensor>& tens, std::vector<const uint16_t*>& gtab) {
+    const int K = set->num_grads;
+    tens.resize(set->ntensors);
+    gtab.assign((size_t)set->ntensors * K, nullptr);
+    for (int ti = 0; ti < set->ntensors; ti++) {
+        const neox_tensor& d = set->tensors[ti];
+        MtTensor& T = tens[ti];
+        T = MtTensor{};
+        T.numel = d.numel;
+        T.wd = d.weight_decay;
+        T.gbase = ti * K;
+        if (!finite(d.weight_decay)) return "tensor " + std::to_string(ti) + ": weight decay must be finite";
+        if (d.numel == 0) continue;
+        if (!d.master || !d.exp_avg || !d.exp_avg_sq || !d.params || !d.grads)
+            return "tensor " + std::to_string(ti) + ": master/exp_avg/exp_avg_sq/params/grads must be non-NULL";
+        if (((uintptr_t)d.master | (uintptr_t)d.exp_avg | (uintptr_t)d.exp_avg_sq) & 3u)
+            return "tensor " + std::to_string(ti) + ": FP32 arrays must be 4-byte aligned";
+        if ((uintptr_t)d.params & 1u) return "tensor " + std::to_string(ti) + ": params must be 2-byte aligned";
+        uintptr_t a16[kMaxGrads + 1];
+        for (int k = 0; k < K; k++) {
+            if (!d.grads[k] || ((uintptr_t)d.grads[k] & 1u))
+                return "tensor " + std::to_string(ti) + ": grads[" + std::to_string(k) + "] NULL or misaligned";
+            gtab[(size_t)ti * K + k] = static_cast<const uint16_t*>(d.grads[k]);
+            a16[k] = (uintptr_t)d.grads[k];
+        }
+        a16[K] = (uintptr_t)d.params;
+        const uintptr_t a32[3] = {(uintptr_t)d.master, (uintptr_t)d.exp_avg, (uintptr_t)d.exp_avg_sq};
+        int vec = 1;
+        const Layout L = choose_layout(d.numel, a16, K + 1, a32, 3, vec);
+        T.master = d.master;
+        T.m = d.exp_avg;
+        T.v = d.exp_avg_sq;
+        T.w = static_cast<uint16_t*>(d.params);
+        T.head = L.head;
+        T.nvec = L.nvec;
+        T.tail0 = L.tail0;
+        T.vec = vec;
+    }
+    return "";
+}
+
+// Resident-grid size for the multi-tensor kernels (at most enough blocks to
+// cover the largest tensor once).
+template <class Kern>
+int mt_grid(Kern kernel, int threads, unsigned long long max_vecs, int sm_count, int cap) {
+    unsigned long long g = (unsigned long long)sm_count * occupancy(kernel, threads);
+    const unsigned long long want = (max_vecs + threads - 1) / threads;
+    if (g > want) g = want;
+    if (g > (unsigned long long)cap) g = cap;
+    return g < 1 ? 1 : (int)g;
+}
+
+neox_status mt_enqueue(neox_multi* h, float lr, const float* lr_dev, cudaStream_t st, bool device_bc,
+                       neox_step_result* result) {
+    if (!lr_dev && (!finite(lr) || lr < 0.0f)) return mfail(h, NEOX_ERR_INVALID_ARGUMENT, "lr must be finite and >= 0");
+    if (result && ((uintptr_t)result & 7u)) return mfail(h, NEOX_ERR_INVALID_ARGUMENT, "result must be 8-byte aligned");
+    if (lr_dev && ((uintptr_t)lr_dev & 3u)) return mfail(h, NEOX_ERR_INVALID_ARGUMENT, "lr_device must be 4-byte aligned");
+    ScalerArgs sa{};
+    sa.post = (double)h->K / (double)h->hp.predivide;
+    sa.inv_pre = (float)(1.0 / (double)h->hp.predivide);
+    sa.clip = h->hp.clip_norm;
+    sa.factor = h->hp.scale_factor;
+    sa.min_scale = h->hp.min_scale;
+    sa.window = h->hp.scale_window;
+    sa.device_bc = device_bc ? 1 : 0;
+    sa.lr = lr;
+    sa.beta1 = h->hp.beta1;
+    sa.beta2 = h->hp.beta2;
+    sa.lr_ptr = lr_dev;
+    sa.result = result;
+    AdamArgs a{};
+    a.lr = lr;
+    a.b1 = h->hp.beta1;
+    a.b2 = h->hp.beta2;
+    a.omb1 = 1.0f - h->hp.beta1;
+    a.omb2 = 1.0f - h->hp.beta2;
+    a.eps = h->hp.eps;
+    if (!device_bc) {
+        const double t1 = (double)(h->t + 1);
+        const double bc1 = 1.0 - std::pow((double)h->hp.beta1, t1);
+        const double bc2 = 1.0 - std::pow((double)h->hp.beta2, t1);
+        a.step_size = (float)((double)lr / bc1);
+        a.bcs = (float)std::sqrt(bc2);
+    }
+    a.device_bc = device_bc ? 1 : 0;
+    a.inv_pre = sa.inv_pre;
+    a.post = sa.post;
+
+    cudaError_t e;
+    {
+        auto k1 = h->gdtype == NEOX_FP16 ? mt_stats_kernel<F16> : mt_stats_kernel<BF16>;
+        const int grid = mt_grid(k1, kMtThreads1, h->max_vecs, h->sm_count, h->max_parts);
+        k1<<<grid, kMtThreads1, 0, st>>>(h->d_tens, h->ntensors, h->d_gtab, h->K, sa, h->d_part_s, h->d_part_b,
+                                         h->d_sc);
+        if ((e = cudaGetLastError()) != cudaSuccess) return mcuda_fail(h, e, "pass-1 launch");
+    }
+    if (h->numel > 0) {
+        auto k2 = h->gdtype == NEOX_FP16 ? (h->wdtype == NEOX_FP16 ? mt_adam_kernel<F16, F16> : mt_adam_kernel<F16, BF16>)
+                                         : (h->wdtype == NEOX_FP16 ? mt_adam_kernel<BF16, F16> : mt_adam_kernel<BF16, BF16>);
+        const int grid = h->grid2;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(kMtThreads3);
+        cfg.dynamicSmemBytes = sizeof(MtTensor) * kMtDescBatch3;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const MtTensor* tens = h->d_tens;
+        const uint16_t* const* gtab = h->d_gtab;
+        const DevScalars* sc = h->d_sc;
+        if ((e = cudaLaunchKernelEx(&cfg, k2, tens, h->ntensors, gtab, h->K, a, sc)) != cudaSuccess)
+            return mcuda_fail(h, e, "pass-2 launch");
+    }
+    return NEOX_OK;
+}
+
+neox_status mt_refresh(neox_multi* h) {
+    if (!h->async_used) return NEOX_OK;
+    DeviceGuard g(h->device);
+    cudaError_t e;
+    if ((e = cudaDeviceSynchronize()) != cudaSuccess) return mcuda_fail(h, e, "waiting for asynchronous steps");
+    DevScalars r;
+    if ((e = cudaMemcpy(&r, h->d_sc, sizeof(r), cudaMemcpyDeviceToHost)) != cudaSuccess)
+        return mcuda_fail(h, e, "reading the device scaler state");
+    h->scale = r.scale;
+    h->good = r.good;
+    h->t = r.t;
+    return NEOX_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+neox_status neox_multi_create(const neox_tensor_set* set, const neox_hparams* hp, int device, neox_multi** out) {
+    g_multi_create_error.clear();
+    if (!out) return mfail(nullptr, NEOX_ERR_INVALID_ARGUMENT, "out is NULL");
+    if (!set) return mfail(nullptr, NEOX_ERR_INVALID_ARGUMENT, "tensor set is NULL");
+    if (const char* why = check_hparams(hp)) return mfail(nullptr, NEOX_ERR_INVALID_ARGUMENT, why);
+    if (set->ntensors < 0 || (set->ntensors > 0 && !set->tensors))
+        return mfail(nullptr, NEOX_ERR_INVALID_ARGUMENT, "ntensors must be >= 0 with a tensor array");
+    if (set->num_grads < 1 || set->num_grads > kMaxGrads)
+        return mfail(nullptr, NEOX_ERR_INVALID_ARGUMENT, "num_grads must be in [1, 64]");
+    if ((set->wdtype != NEOX_FP16 && set->wdtype != NEOX_BF16) || (set->gdtype != NEOX_FP16 && set->gdtype != NEOX_BF16))
+        return mfail(nullptr, NEOX_ERR_INVALID_ARGUMENT, "dtype must be NEOX_FP16 or NEOX_BF16");
+    std::vector<MtTensor> tens;
+    std::vector<const uint16_t*> gtab;
+    const std::string why = build_tables(set, tens, gtab);
+    if (!why.empty()) return mfail(nullptr, NEOX_ERR_INVALID_ARGUMENT, why);
+
+    auto* h = new (std::nothrow) neox_multi();
+    if (!h) return mfail(nullptr, NEOX_ERR_OUT_OF_MEMORY, "host allocation failed");
+    h->device = device;
+    h->ntensors = set->ntensors;
+    h->K = set->num_grads;
+    h->wdtype = set->wdtype;
+    h->gdtype = set->gdtype;
+    h->hp = *hp;
+    h->scale = hp->init_scale;
+    for (const auto& T : tens) {
+        h->numel += T.numel;
+        if (T.nvec > h->max_vecs) h->max_vecs = T.nvec;
+    }
+    h->tens = tens;
+    neox_status st = NEOX_OK;
+    cudaError_t e;
+    {
+        int ndev = 0;
+        if ((e = cudaGetDeviceCount(&ndev)) != cudaSuccess) { st = mcuda_fail(nullptr, e, "cudaGetDeviceCount"); goto done; }
+        if (device < 0 || device >= ndev) { st = mfail(nullptr, NEOX_ERR_INVALID_ARGUMENT, "no such CUDA device"); goto done; }
+        DeviceGuard g(device);
+        if (!g.ok) { st = mfail(nullptr, NEOX_ERR_CUDA, "cudaSetDevice failed"); goto done; }
+        int major = 0;
+        if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&h->sm_count, cudaDevAttrMultiProcessorCount, device)) != cudaSuccess) {
+            st = mcuda_fail(nullptr, e, "cudaDeviceGetAttribute");
+            goto done;
+        }
+        if (major != 10) { st = mfail(nullptr, NEOX_ERR_UNSUPPORTED, "this library is built for sm_100a (B200)"); goto done; }
+        h->max_parts = h->sm_count * kMaxBlocksPerSm;
+        const size_t nt = tens.size() ? tens.size() : 1, ng = gtab.size() ? gtab.size() : 1;
+        if ((e = cudaMalloc(&h->d_tens, sizeof(MtTensor) * nt)) != cudaSuccess ||
+            (e = cudaMalloc((void**)&h->d_gtab, sizeof(void*) * ng)) != cudaSuccess ||
+            (e = cudaMalloc(&h->d_sc, sizeof(DevScalars))) != cudaSuccess ||
+            (e = cudaMalloc(&h->d_part_s, sizeof(double) * h->max_parts)) != cudaSuccess ||
+            (e = cudaMalloc(&h->d_part_b, sizeof(int) * h->max_parts)) != cudaSuccess ||
+            (e = cudaMallocHost(&h->h_sc, sizeof(DevScalars))) != cudaSuccess) {
+            st = mcuda_fail(nullptr, e, "allocation");
+            goto done;
+        }
+        if ((!tens.empty() && (e = cudaMemcpy(h->d_tens, tens.data(), sizeof(MtTensor) * tens.size(),
+                                              cudaMemcpyHostToDevice)) != cudaSuccess) ||
+            (!gtab.empty() && (e = cudaMemcpy(h->d_gtab, gtab.data(), sizeof(void*) * gtab.size(),
+                                              cudaMemcpyHostToDevice)) != cudaSuccess)) {
+            st = mcuda_fail(nullptr, e, "copying the tensor tables");
+            goto done;
+        }
+        DevScalars init{};
+        init.scale = hp->init_scale;
+        init.scale_used = hp->init_scale;
+        if ((e = cudaMemcpy(h->d_sc, &init, sizeof(init), cudaMemcpyHostToDevice)) != cudaSuccess) {
+            st = mcuda_fail(nullptr, e, "cudaMemcpy scalars");
+            goto done;
+        }
+        // pass 2 runs with kMtDescBatch3 descriptors of dynamic shared memory
+        auto k2 = h->gdtype == NEOX_FP16 ? (h->wdtype == NEOX_FP16 ? mt_adam_kernel<F16, F16> : mt_adam_kernel<F16, BF16>)
+                                         : (h->wdtype == NEOX_FP16 ? mt_adam_kernel<BF16, F16> : mt_adam_kernel<BF16, BF16>);
+        const int dyn = (int)(sizeof(MtTensor) * kMtDescBatch3);
+        int occ = 0;
+        if ((e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn)) != cudaSuccess ||
+            (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k2, kMtThreads3, dyn)) != cudaSuccess) {
+            st = mcuda_fail(nullptr, e, "configuring the update kernel");
+            goto done;
+        }
+        unsigned long long g2 = (unsigned long long)h->sm_count * (occ < 1 ? 1 : occ);
+        const unsigned long long want2 = (h->max_vecs + kMtThreads3 - 1) / kMtThreads3;
+        if (g2 > want2) g2 = want2;
+        h->grid2 = g2 < 1 ? 1 : (int)g2;
+    }
+done:
+    if (st != NEOX_OK) {
+        DeviceGuard g(device);
+        mfree(h);
+        delete h;
+        return st;
+    }
+    *out = h;
+    return NEOX_OK;
+}
+
+void neox_multi_destroy(neox_multi* h) {
+    if (!h) return;
+    {
+        DeviceGuard g(h->device);
+        mfree(h);
+    }
+    delete h;
+}
+
+const char* neox_multi_last_error(const neox_multi* h) {
+    return h ? h->last_error.c_str() : g_multi_create_error.c_str();
+}
+
+neox_status neox_multi_rebind_grads(neox_multi* h, const void* const* grads) {
+    if (!h) return NEOX_ERR_INVALID_ARGUMENT;
+    if (!grads && h->ntensors > 0) return mfail(h, NEOX_ERR_INVALID_ARGUMENT, "grads is NULL");
+    std::vector<const uint16_t*> gtab((size_t)h->ntensors * h->K, nullptr);
+    for (int ti = 0; ti < h->ntensors; ti++) {
+        const MtTensor& T = h->tens[ti];
+        if (T.numel == 0) continue;
+        for (int k = 0; k < h->K; k++) {
+            const void* p = grads[(size_t)ti * h->K + k];
+            // the new pointers must keep the tensor's vector layout
+            const int al = 2 * T.vec;
+            if (!p || (((uintptr_t)p + 2 * T.head) % al) != 0 || ((uintptr_t)p & 1u))
+                return mfail(h, NEOX_ERR_INVALID_ARGUMENT,
+                             "tensor " + std::to_string(ti) + ": grads[" + std::to_string(k) +
+                                 "] NULL or with another alignment than at create");
+            gtab[(size_t)ti * h->K + k] = static_cast<const uint16_t*>(p);
+        }
+    }
+    DeviceGuard g(h->device);
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess && !gtab.empty())
+        e = cudaMemcpy(h->d_gtab, gtab.data(), sizeof(void*) * gtab.size(), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return mcuda_fail(h, e, "updating the gradient table");
+    return NEOX_OK;
+}
+
+neox_status neox_multi_step(neox_multi* h, float lr, void* cuda_stream, neox_step_result* out) {
+    if (!h) return NEOX_ERR_INVALID_ARGUMENT;
+    h->last_error.clear();
+    if (!out) return mfail(h, NEOX_ERR_INVALID_ARGUMENT, "out is NULL");
+    DeviceGuard g(h->device);
+    if (!g.ok) return mfail(h, NEOX_ERR_CUDA, "cudaSetDevice failed");
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    if (neox_status s = mt_enqueue(h, lr, nullptr, st, h->async_used, nullptr); s != NEOX_OK) return s;
+    cudaError_t e;
+    if ((e = cudaMemcpyAsync(h->h_sc, h->d_sc, sizeof(DevScalars), cudaMemcpyDeviceToHost, st)) != cudaSuccess)
+        return mcuda_fail(h, e, "cudaMemcpyAsync result");
+    if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return mcuda_fail(h, e, "step execution");
+    const DevScalars& r = *h->h_sc;
+    out->overflow = r.overflow;
+    out->grad_norm = r.norm;
+    out->clip_coef = r.coef;
+    out->loss_scale = r.scale_used;
+    out->loss_scale_next = r.scale;
+    out->good_steps = r.good;
+    out->applied_steps = r.t;
+    h->scale = r.scale;
+    h->good = r.good;
+    h->t = r.t;
+    return NEOX_OK;
+}
+
+neox_status neox_multi_step_async(neox_multi* h, float lr, const float* lr_device, void* cuda_stream,
+                                  neox_step_result* result) {
+    if (!h) return NEOX_ERR_INVALID_ARGUMENT;
+    h->last_error.clear();
+    DeviceGuard g(h->device);
+    if (!g.ok) return mfail(h, NEOX_ERR_CUDA, "cudaSetDevice failed");
+    h->async_used = true;
+    return mt_enqueue(h, lr, lr_device, static_cast<cudaStream_t>(cuda_stream), true, result);
+}
+
+neox_status neox_multi_set_hparams(neox_multi* h, const neox_hparams* hp) {
+    if (!h) return NEOX_ERR_INVALID_ARGUMENT;
+    if (const char* why = check_hparams(hp)) return mfail(h, NEOX_ERR_INVALID_ARGUMENT, why);
+    h->hp = *hp;
+    return NEOX_OK;
+}
+
+neox_status neox_multi_get_state(const neox_multi* h, float* scale, int32_t* good, int64_t* t) {
+    if (!h) return NEOX_ERR_INVALID_ARGUMENT;
+    if (neox_status s = mt_refresh(const_cast<neox_multi*>(h)); s != NEOX_OK) return s;
+    if (scale) *scale = h->scale;
+    if (good) *good = h->good;
+    if (t) *t = h->t;
+    return NEOX_OK;
+}
+
+neox_status neox_multi_set_state(neox_multi* h, float scale, int32_t good, int64_t t) {
+    if (!h) return NEOX_ERR_INVALID_ARGUMENT;
+    if (!(scale > 0.0f) || !finite(scale) || good < 0 || t < 0)
+        return mfail(h, NEOX_ERR_INVALID_ARGUMENT, "state needs a finite scale > 0, good >= 0, t >= 0");
+    DeviceGuard g(h->device);
+    cudaError_t e = cudaSuccess;
+    if (h->async_used) e = cudaDeviceSynchronize();
+    DevScalars s{};
+    s.scale = scale;
+    s.scale_used = scale;
+    s.good = good;
+    s.t = t;
+    if (e == cudaSuccess) e = cudaMemcpy(h->d_sc, &s, sizeof(s), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return mcuda_fail(h, e, "writing the scaler state");
+    h->scale = scale;
+    h->good = good;
+    h->t = t;
+    return NEOX_OK;
+}
+
+}  // extern "C"

@@ -32,6 +32,7 @@
 // a sequential FP32 evaluation.
 
 #include "neox_shard.h"
+#include "neox_common.cuh"
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -45,264 +46,6 @@
 
 namespace {
 
-constexpr int kMaxGrads = 64;
-constexpr int kThreads1 = 512;   // pass-1 block
-constexpr int kUnroll1 = 4;      // pass-1 vectors in flight per thread
-constexpr int kThreads3 = 256;   // pass-2 block
-constexpr int kUnroll3 = 1;      // pass-2 vectors in flight per thread
-constexpr int kMaxBlocksPerSm = 32;
-
-struct GradPtrs {
-    const uint16_t* p[kMaxGrads];
-};
-
-// Device-resident scalars of one shard (64 bytes).  `scale`, `good`, `t` are
-// the scaler / step state; the rest describe the most recent step.
-struct __align__(64) DevScalars {
-    double sumsq;          // sum of squared unscaled grads of the last step
-    float scale;           // S the next step's grads carry
-    int32_t good;          // consecutive applied steps
-    long long t;           // applied steps
-    int32_t overflow;      // last step overflowed
-    float coef;            // clip coefficient of the last step
-    float scale_used;      // S the last step's grads carried
-    float norm;            // pre-clip norm of the last step (+inf on overflow)
-    unsigned int blocks_done;  // pass-1 ticket counter, back to 0 after each step
-    float step_size;       // device-computed fl32(lr / bc1) of the last step (asynchronous steps)
-    float bc2_sqrt;        // device-computed fl32(sqrt(bc2)) of the last step (asynchronous steps)
-    float lr;              // learning rate of the last step (asynchronous steps)
-    int32_t pad_[2];
-};
-static_assert(sizeof(DevScalars) == 64, "DevScalars is one 64-byte block");
-
-// Which elements use vectors: [0, head) scalar, [head, head + nvec*VEC)
-// vectors of VEC, [tail0, n) scalar.
-struct Layout {
-    unsigned long long n, head, nvec, tail0;
-};
-
-struct ScalerArgs {
-    double post;          // K / predivide
-    float inv_pre;        // fl32(1 / predivide)
-    float clip;           // <= 0: off
-    float factor, min_scale;
-    int32_t window;
-    // asynchronous steps: the bias corrections are formed on the device from
-    // the device step count, and the result is written to `result`
-    int32_t device_bc;
-    float lr, beta1, beta2;
-    const float* lr_ptr;       // when non-NULL, the learning rate is read here
-    neox_step_result* result;  // device-accessible; NULL = not written
-};
-
-struct AdamArgs {
-    float lr, b1, b2, omb1, omb2, eps;
-    float step_size;      // fl32(lr / bc1) for t+1
-    float bcs;            // fl32(sqrt(bc2)) for t+1
-    float inv_pre;
-    int32_t device_bc;    // take lr, step_size and bcs from the device scalars
-    double post;
-};
-
-// ---------------------------------------------------------------- 16-bit types
-struct F16 {
-    static __device__ __forceinline__ float dec(uint16_t h) { return __half2float(__ushort_as_half(h)); }
-    static __device__ __forceinline__ uint16_t enc(float f) { return __half_as_ushort(__float2half_rn(f)); }
-    static __device__ __forceinline__ uint32_t enc2(float lo, float hi) {
-        __half2 h = __floats2half2_rn(lo, hi);
-        return *reinterpret_cast<uint32_t*>(&h);
-    }
-};
-struct BF16 {
-    static __device__ __forceinline__ float dec(uint16_t h) { return __uint_as_float(uint32_t(h) << 16); }
-    static __device__ __forceinline__ uint16_t enc(float f) { return __bfloat16_as_ushort(__float2bfloat16_rn(f)); }
-    static __device__ __forceinline__ uint32_t enc2(float lo, float hi) {
-        __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-        return *reinterpret_cast<uint32_t*>(&h);
-    }
-};
-
-// ---------------------------------------------------------------- vector I/O
-// VEC 16-bit values starting at p (aligned to 2*VEC bytes), read-only data.
-template <int VEC>
-__device__ __forceinline__ void ld16(const uint16_t* p, uint16_t (&o)[VEC]) {
-    if constexpr (VEC == 8) {
-        uint4 r = __ldcs(reinterpret_cast<const uint4*>(p));
-        uint32_t w[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-        for (int i = 0; i < 4; i++) { o[2 * i] = uint16_t(w[i]); o[2 * i + 1] = uint16_t(w[i] >> 16); }
-    } else if constexpr (VEC == 4) {
-        uint2 r = __ldcs(reinterpret_cast<const uint2*>(p));
-        o[0] = uint16_t(r.x); o[1] = uint16_t(r.x >> 16); o[2] = uint16_t(r.y); o[3] = uint16_t(r.y >> 16);
-    } else if constexpr (VEC == 2) {
-        uint32_t r = __ldcs(reinterpret_cast<const unsigned int*>(p));
-        o[0] = uint16_t(r); o[1] = uint16_t(r >> 16);
-    } else {
-        o[0] = __ldcs(reinterpret_cast<const unsigned short*>(p));
-    }
-}
-
-template <class W, int VEC>
-__device__ __forceinline__ void st16(uint16_t* p, const float (&x)[VEC]) {
-    if constexpr (VEC == 8) {
-        uint4 r = make_uint4(W::enc2(x[0], x[1]), W::enc2(x[2], x[3]), W::enc2(x[4], x[5]), W::enc2(x[6], x[7]));
-        __stcs(reinterpret_cast<uint4*>(p), r);
-    } else if constexpr (VEC == 4) {
-        uint2 r = make_uint2(W::enc2(x[0], x[1]), W::enc2(x[2], x[3]));
-        __stcs(reinterpret_cast<uint2*>(p), r);
-    } else if constexpr (VEC == 2) {
-        __stcs(reinterpret_cast<unsigned int*>(p), W::enc2(x[0], x[1]));
-    } else {
-        __stcs(reinterpret_cast<unsigned short*>(p), W::enc(x[0]));
-    }
-}
-
-// VEC FP32 values at p (16-byte aligned when VEC >= 4).
-template <int VEC>
-__device__ __forceinline__ void ld32(const float* p, float (&o)[VEC]) {
-    if constexpr (VEC >= 4) {
-#pragma unroll
-        for (int q = 0; q < VEC / 4; q++) {
-            float4 r = __ldcs(reinterpret_cast<const float4*>(p) + q);
-            o[4 * q] = r.x; o[4 * q + 1] = r.y; o[4 * q + 2] = r.z; o[4 * q + 3] = r.w;
-        }
-    } else if constexpr (VEC == 2) {
-        float2 r = __ldcs(reinterpret_cast<const float2*>(p));
-        o[0] = r.x; o[1] = r.y;
-    } else {
-        o[0] = __ldcs(p);
-    }
-}
-
-template <int VEC>
-__device__ __forceinline__ void st32(float* p, const float (&x)[VEC]) {
-    if constexpr (VEC >= 4) {
-#pragma unroll
-        for (int q = 0; q < VEC / 4; q++)
-            __stcs(reinterpret_cast<float4*>(p) + q, make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]));
-    } else if constexpr (VEC == 2) {
-        __stcs(reinterpret_cast<float2*>(p), make_float2(x[0], x[1]));
-    } else {
-        __stcs(p, x[0]);
-    }
-}
-
-__device__ __forceinline__ bool not_finite(float x) {
-    return (__float_as_uint(x) & 0x7f800000u) == 0x7f800000u;
-}
-
-// Unscaled gradients of VEC consecutive elements from global index i:
-// a = sum_k fl32(g_k * inv_pre) in buffer order (starting from +0, as a
-// sequential sum does), then fl32(a * inv_us).
-template <class G, int VEC>
-__device__ __forceinline__ void ingest(const GradPtrs& gp, int K, unsigned long long i,
-                                       float inv_pre, float inv_us, float (&g)[VEC]) {
-#pragma unroll
-    for (int e = 0; e < VEC; e++) g[e] = 0.0f;
-    const bool pre1 = inv_pre == 1.0f;  // x * 1 == x exactly: skip the multiply
-    for (int k = 0; k < K; k++) {
-        uint16_t h[VEC];
-        ld16<VEC>(gp.p[k] + i, h);
-        if (pre1) {
-#pragma unroll
-            for (int e = 0; e < VEC; e++) g[e] = __fadd_rn(g[e], G::dec(h[e]));
-        } else {
-#pragma unroll
-            for (int e = 0; e < VEC; e++) g[e] = __fadd_rn(g[e], __fmul_rn(G::dec(h[e]), inv_pre));
-        }
-    }
-#pragma unroll
-    for (int e = 0; e < VEC; e++) g[e] = __fmul_rn(g[e], inv_us);
-}
-
-// U vectors at global indices i0, i0 + di, ..., ingested together: for every
-// buffer the U loads are issued before any of them is used, so each thread
-// keeps U 16-byte requests in flight.  Per element the arithmetic (and its
-// order over buffers) is that of ingest().
-template <class G, int VEC, int U>
-__device__ __forceinline__ void ingest_batch(const GradPtrs& gp, int K, unsigned long long i0, unsigned long long di,
-                                             float inv_pre, float inv_us, float (&g)[U][VEC]) {
-#pragma unroll
-    for (int u = 0; u < U; u++)
-#pragma unroll
-        for (int e = 0; e < VEC; e++) g[u][e] = 0.0f;
-    const bool pre1 = inv_pre == 1.0f;  // x * 1 == x exactly: skip the multiply
-    for (int k = 0; k < K; k++) {
-        uint16_t h[U][VEC];
-#pragma unroll
-        for (int u = 0; u < U; u++) ld16<VEC>(gp.p[k] + i0 + u * di, h[u]);
-        if (pre1) {
-#pragma unroll
-            for (int u = 0; u < U; u++)
-#pragma unroll
-                for (int e = 0; e < VEC; e++) g[u][e] = __fadd_rn(g[u][e], G::dec(h[u][e]));
-        } else {
-#pragma unroll
-            for (int u = 0; u < U; u++)
-#pragma unroll
-                for (int e = 0; e < VEC; e++) g[u][e] = __fadd_rn(g[u][e], __fmul_rn(G::dec(h[u][e]), inv_pre));
-        }
-    }
-#pragma unroll
-    for (int u = 0; u < U; u++)
-#pragma unroll
-        for (int e = 0; e < VEC; e++) g[u][e] = __fmul_rn(g[u][e], inv_us);
-}
-
-__device__ __forceinline__ float unscale_factor(double post, float scale) {
-    return (float)(1.0 / (post * (double)scale));
-}
-
-// Sum of squares of a vector (FP32 within the vector) and the non-finite
-// flag.  A sum of squares is finite exactly when every element is finite and
-// no square or partial sum passes FP32's range, so one test per vector
-// replaces a test per element; only a vector that fails it looks at its
-// elements (and, when they are all finite, redoes the sum in FP64).
-template <int VEC>
-__device__ __forceinline__ double vec_sumsq(const float (&g)[VEC], int& bad) {
-    float q = 0.0f;
-#pragma unroll
-    for (int e = 0; e < VEC; e++) q = __fmaf_rn(g[e], g[e], q);
-    if (!(q <= 3.40282346638528859812e+38f)) {
-        int vb = 0;
-#pragma unroll
-        for (int e = 0; e < VEC; e++) vb |= not_finite(g[e]);
-        bad |= vb;
-        if (!vb) {
-            double d = 0.0;
-#pragma unroll
-            for (int e = 0; e < VEC; e++) d += (double)g[e] * (double)g[e];
-            return d;
-        }
-    }
-    return (double)q;
-}
-
-// Block-wide reduction of (double, int-or) with a fixed shape.
-template <int THREADS>
-__device__ __forceinline__ void block_reduce(double& s, int& bad, double* sh_s, int* sh_b) {
-    const unsigned full = 0xffffffffu;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        s += __shfl_down_sync(full, s, off);
-        bad |= __shfl_down_sync(full, bad, off);
-    }
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (lane == 0) { sh_s[warp] = s; sh_b[warp] = bad; }
-    __syncthreads();
-    if (warp == 0) {
-        constexpr int NW = THREADS / 32;
-        s = lane < NW ? sh_s[lane] : 0.0;
-        bad = lane < NW ? sh_b[lane] : 0;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            s += __shfl_down_sync(full, s, off);
-            bad |= __shfl_down_sync(full, bad, off);
-        }
-    }
-}
-
-// ---------------------------------------------------------------- pass 1
 // The vector loop of pass 1.  KFIX = 1 compiles the single-buffer case with
 // K known to be 1; KFIX = 0 takes K at run time.
 template <class G, int VEC, bool WRITE_ACC, int KFIX>
@@ -359,90 +102,7 @@ grad_stats_kernel(GradPtrs gp, int K, Layout L, ScalerArgs sa, float* __restrict
         }
     }
 
-    // Let the update kernel's blocks start their prologue as this grid winds
-    // down; they wait (griddepcontrol.wait) for this grid's completion before
-    // reading anything it writes.
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    block_reduce<kThreads1>(s, bad, sh_s, sh_b);
-    if (threadIdx.x == 0) {
-        part_s[blockIdx.x] = s;
-        part_b[blockIdx.x] = bad;
-        __threadfence();
-        const unsigned ticket = atomicAdd(&sc->blocks_done, 1u);
-        is_last = (ticket == gridDim.x - 1);
-    }
-    __syncthreads();
-    if (!is_last) return;
-
-    // Last block: every other block's partial is visible (each fenced before
-    // taking its ticket).  Reduce them in a fixed order.
-    __threadfence();
-    s = 0.0;
-    bad = 0;
-    for (unsigned j = threadIdx.x; j < gridDim.x; j += kThreads1) {
-        s += __ldcg(part_s + j);
-        bad |= __ldcg(part_b + j);
-    }
-    __syncthreads();
-    block_reduce<kThreads1>(s, bad, sh_s, sh_b);
-    if (threadIdx.x != 0) return;
-
-    // Scalar decisions of the step.
-    int overflow = bad != 0;
-    const double norm = sqrt(s);
-    if (!overflow && !isfinite(norm)) overflow = 1;
-    float S = sc->scale;
-    int good = sc->good;
-    long long t = sc->t;
-    sc->scale_used = S;
-    sc->sumsq = s;
-    sc->overflow = overflow;
-    if (overflow) {
-        const float d = S / sa.factor;
-        S = d > sa.min_scale ? d : sa.min_scale;
-        good = 0;
-        sc->coef = 0.0f;
-        sc->norm = __int_as_float(0x7f800000);
-    } else {
-        good += 1;
-        if (good >= sa.window) {
-            const float u = S * sa.factor;
-            if (!not_finite(u)) S = u;
-            good = 0;
-        }
-        t += 1;
-        float c = 1.0f;
-        if (sa.clip > 0.0f) {
-            const double cd = (double)sa.clip / (norm + 1e-6);
-            if (cd < 1.0) c = (float)cd;
-        }
-        sc->coef = c;
-        sc->norm = (float)norm;
-    }
-    sc->scale = S;
-    sc->good = good;
-    sc->t = t;
-    if (sa.device_bc) {
-        const float lr = sa.lr_ptr ? *sa.lr_ptr : sa.lr;
-        sc->lr = lr;
-        if (!overflow) {
-            const double bc1 = 1.0 - pow((double)sa.beta1, (double)t);
-            const double bc2 = 1.0 - pow((double)sa.beta2, (double)t);
-            sc->step_size = (float)((double)lr / bc1);
-            sc->bc2_sqrt = (float)sqrt(bc2);
-        }
-        if (sa.result) {
-            neox_step_result* r = sa.result;
-            r->overflow = overflow;
-            r->grad_norm = sc->norm;
-            r->clip_coef = sc->coef;
-            r->loss_scale = sc->scale_used;
-            r->loss_scale_next = S;
-            r->good_steps = good;
-            r->applied_steps = t;
-        }
-    }
-    sc->blocks_done = 0;
+    finish_pass1<kThreads1>(s, bad, part_s, part_b, sc, sa, sh_s, sh_b, &is_last);
 }
 
 // ---------------------------------------------------------------- pass 2
@@ -463,25 +123,6 @@ __device__ __forceinline__ void seg_seek(SegCursor& c, unsigned long long i, con
     c.seg = lo;
     c.end = __ldg(seg_end + lo);
     c.keep = __fsub_rn(1.0f, __fmul_rn(lr, __ldg(seg_wd + lo)));
-}
-
-template <int VEC>
-__device__ __forceinline__ void adam_vec(const float (&g)[VEC], const float (&keep)[VEC], float c,
-                                         const AdamArgs& a, float (&p)[VEC], float (&m)[VEC], float (&v)[VEC]) {
-#pragma unroll
-    for (int e = 0; e < VEC; e++) {
-        const float gh = __fmul_rn(g[e], c);
-        const float mj = __fadd_rn(__fmul_rn(a.b1, m[e]), __fmul_rn(a.omb1, gh));
-        const float gg = __fmul_rn(a.omb2, gh);
-        const float vj = __fadd_rn(__fmul_rn(a.b2, v[e]), __fmul_rn(gg, gh));
-        const float den = __fadd_rn(__fdiv_rn(__fsqrt_rn(vj), a.bcs), a.eps);
-        float pj = __fmul_rn(p[e], keep[e]);
-        const float upd = __fdiv_rn(mj, den);
-        pj = __fsub_rn(pj, __fmul_rn(a.step_size, upd));
-        m[e] = mj;
-        v[e] = vj;
-        p[e] = pj;
-    }
 }
 
 // The vector loop of pass 2 (KFIX as in pass1_vectors).
@@ -634,7 +275,7 @@ struct neox_shard {
     unsigned long long* d_seg_end = nullptr;
     float* d_seg_wd = nullptr;
     int nsegs = 0;
-    float* d_acc = nullptr;  // FP32 sum of K >= 5 buffers (numel + 4 floats)
+    float* d_acc = nullptr;  // FP32 sum of K >= 5 buffers (numel + 32 floats)
     DevScalars* h_sc = nullptr;  // pinned result slot
     unsigned long long owned_bytes = 0;
     // profiling
@@ -649,19 +290,6 @@ namespace {
 
 thread_local std::string g_create_error;
 
-struct DeviceGuard {
-    int prev = -1;
-    bool ok = true;
-    explicit DeviceGuard(int dev) {
-        if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
-        if (prev != dev) ok = cudaSetDevice(dev) == cudaSuccess;
-    }
-    ~DeviceGuard() {
-        int cur = -1;
-        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
-    }
-};
-
 neox_status fail(neox_shard* h, neox_status st, const std::string& msg) {
     if (h) h->last_error = msg; else g_create_error = msg;
     return st;
@@ -670,73 +298,6 @@ neox_status fail(neox_shard* h, neox_status st, const std::string& msg) {
 neox_status cuda_fail(neox_shard* h, cudaError_t e, const char* what) {
     std::string msg = std::string(what) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")";
     return fail(h, e == cudaErrorMemoryAllocation ? NEOX_ERR_OUT_OF_MEMORY : NEOX_ERR_CUDA, msg);
-}
-
-bool finite(float x) { return std::isfinite(x); }
-
-const char* check_hparams(const neox_hparams* hp) {
-    if (!hp) return "hparams is NULL";
-    if (!(hp->beta1 >= 0.0f && hp->beta1 < 1.0f)) return "beta1 must be in [0, 1)";
-    if (!(hp->beta2 >= 0.0f && hp->beta2 < 1.0f)) return "beta2 must be in [0, 1)";
-    if (!(hp->eps >= 0.0f) || !finite(hp->eps)) return "eps must be finite and >= 0";
-    if (!finite(hp->clip_norm)) return "clip_norm must be finite";
-    if (!(hp->predivide > 0.0f) || !finite(hp->predivide)) return "predivide must be finite and > 0";
-    if (!(hp->init_scale > 0.0f) || !finite(hp->init_scale)) return "init_scale must be finite and > 0";
-    if (!(hp->scale_factor >= 1.0f) || !finite(hp->scale_factor)) return "scale_factor must be finite and >= 1";
-    if (!(hp->min_scale >= 0.0f) || !finite(hp->min_scale)) return "min_scale must be finite and >= 0";
-    if (hp->scale_window < 1) return "scale_window must be >= 1";
-    return nullptr;
-}
-
-int elem_size(neox_dtype) { return 2; }
-
-// Choose the widest vector (8, 4, 2, 1 elements) and a head h < VEC such that
-// every 16-bit array is 2*VEC-byte aligned and every FP32 array 16-byte (VEC
-// >= 4) or 4*VEC-byte aligned at element h.
-Layout choose_layout(unsigned long long n, const uintptr_t* a16, int n16, const uintptr_t* a32, int n32, int& vec_out) {
-    for (int vec = 8; vec >= 1; vec >>= 1) {
-        const uintptr_t al16 = 2u * vec;
-        const uintptr_t al32 = vec >= 4 ? 16u : 4u * vec;
-        for (int h = 0; h < vec; h++) {
-            bool ok = true;
-            for (int i = 0; i < n16 && ok; i++) ok = ((a16[i] + 2u * h) % al16) == 0;
-            for (int i = 0; i < n32 && ok; i++) ok = ((a32[i] + 4u * h) % al32) == 0;
-            if (!ok) continue;
-            Layout L;
-            L.n = n;
-            L.head = (unsigned long long)h < n ? h : n;
-            L.nvec = (n - L.head) / vec;
-            L.tail0 = L.head + L.nvec * vec;
-            vec_out = vec;
-            return L;
-        }
-    }
-    vec_out = 1;  // unreachable: VEC = 1 always fits
-    return Layout{n, 0, n, n};
-}
-
-// Resident blocks per SM of one kernel instantiation (queried once per
-// instantiation and device; B200 parts are uniform, so the first answer holds).
-template <class K>
-int occupancy(K kernel, int threads) {
-    static int cached = 0;
-    if (cached == 0) {
-        int occ = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, threads, 0) != cudaSuccess || occ < 1) occ = 1;
-        cached = occ;
-    }
-    return cached;
-}
-
-template <class K>
-int grid_for(K kernel, int threads, unsigned long long work_items, int sm_count, int cap) {
-    const int occ = occupancy(kernel, threads);
-    unsigned long long want = (work_items + threads - 1) / threads;
-    unsigned long long full = (unsigned long long)sm_count * (unsigned long long)occ;
-    unsigned long long g = want < full ? want : full;
-    if (g < 1) g = 1;
-    if (g > (unsigned long long)cap) g = cap;
-    return (int)g;
 }
 
 template <class G, int VEC, bool ACC>
@@ -870,8 +431,8 @@ neox_status enqueue_step(neox_shard* h, const void* const* grads, int32_t num_gr
     Layout L = h->numel > 0 ? choose_layout(h->numel, a16, num_grads + 1, a32, 3, vec) : Layout{0, 0, 0, 0};
     float* acc = nullptr;
     if (use_acc) {
-        const unsigned long long hh = L.head % 4;
-        acc = h->d_acc + ((4 - hh) % 4);  // &acc[head] is 16-byte aligned
+        const unsigned long long hh = L.head % 32;
+        acc = h->d_acc + ((32 - hh) % 32);  // &acc[head] sits on a 128-byte line
     }
 
     ScalerArgs sa{};
@@ -1040,8 +601,8 @@ neox_status neox_shard_create(const neox_shard_desc* d, const neox_hparams* hp, 
         if ((e = cudaMalloc(&h->d_seg_wd, sizeof(float) * nsegs)) != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMalloc segments"); goto done; }
         bytes += (sizeof(unsigned long long) + sizeof(float)) * nsegs;
         if (h->max_grads >= 5 && h->numel > 0) {
-            if ((e = cudaMalloc(&h->d_acc, sizeof(float) * (h->numel + 4))) != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMalloc accumulation buffer"); goto done; }
-            bytes += sizeof(float) * (h->numel + 4);
+            if ((e = cudaMalloc(&h->d_acc, sizeof(float) * (h->numel + 32))) != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMalloc accumulation buffer"); goto done; }
+            bytes += sizeof(float) * (h->numel + 32);
         }
         h->owned_bytes = bytes;
         if ((e = cudaMallocHost(&h->h_sc, sizeof(DevScalars))) != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMallocHost"); goto done; }

@@ -117,3 +117,31 @@ def test_null_handle_calls():
     assert L.neox_shard_set_hparams(None, None) == _abi.NEOX_ERR_INVALID_ARGUMENT
     assert L.neox_shard_scratch_bytes(None) == 0
     L.neox_shard_destroy(None)
+
+
+def test_multi_create_rejects_invalid_arguments_before_cuda():
+    L = _abi.lib()
+    h = ctypes.c_void_p()
+    hp = _hp()
+    grads = (ctypes.c_void_p * 1)(4096)
+    good_t = _abi.neox_tensor(16, 0.1, 4096, 8192, 12288, 16384, ctypes.cast(grads, ctypes.POINTER(ctypes.c_void_p)))
+    cases = [
+        (_abi.neox_tensor_set(-1, 1, 0, 0, None), "ntensors"),
+        (_abi.neox_tensor_set(1, 0, 0, 0, ctypes.pointer(good_t)), "num_grads"),
+        (_abi.neox_tensor_set(1, 65, 0, 0, ctypes.pointer(good_t)), "num_grads"),
+        (_abi.neox_tensor_set(1, 1, 5, 0, ctypes.pointer(good_t)), "dtype"),
+        (_abi.neox_tensor_set(1, 1, 0, 0, ctypes.pointer(
+            _abi.neox_tensor(16, 0.1, 4096, 8194, 12288, 16384, ctypes.cast(grads, ctypes.POINTER(ctypes.c_void_p))))),
+         "aligned"),
+        (_abi.neox_tensor_set(1, 1, 0, 0, ctypes.pointer(_abi.neox_tensor(16, 0.1, 4096, 8192, 12288, 16384, None))),
+         "non-NULL"),
+        (_abi.neox_tensor_set(1, 1, 0, 0, ctypes.pointer(
+            _abi.neox_tensor(16, float("nan"), 4096, 8192, 12288, 16384,
+                             ctypes.cast(grads, ctypes.POINTER(ctypes.c_void_p))))), "weight decay"),
+    ]
+    for tset, why in cases:
+        assert L.neox_multi_create(ctypes.byref(tset), ctypes.byref(hp), 0, ctypes.byref(h)) == \
+            _abi.NEOX_ERR_INVALID_ARGUMENT
+        assert why in L.neox_multi_last_error(None).decode()
+    assert L.neox_multi_step(None, 1e-3, None, None) == _abi.NEOX_ERR_INVALID_ARGUMENT
+    L.neox_multi_destroy(None)

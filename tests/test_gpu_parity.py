@@ -312,3 +312,19 @@ def test_huge_finite_gradients_are_not_overflow():
         c.check_result(res, info)
         c.check_state()
     c.close()
+
+
+@pytest.mark.parametrize("max_grads", [64, 1])
+def test_maximum_buffer_count(max_grads):
+    """K = 64 gradient buffers (the largest the ABI takes), pre-divide 64,
+    through the FP32-sum path and the re-read path."""
+    n = 70_001
+    hp = Hparams(clip_norm=1.0, predivide=64.0, init_scale=2.0 ** 8)
+    c = ShardCase(n, K=64, hp=hp, max_grads=max_grads, offsets={"all": 2}, lr=6e-4)
+    for s in range(1, 4):
+        c.gen_normal(s, 1e-3)
+        res, info = c.step()
+        c.check_result(res, info)
+        c.check_state()
+    assert c.guards_intact()
+    c.close()
