@@ -31,7 +31,7 @@ sys.path.insert(0, ROOT)
 METRIC = "Adam shard-step Gparams/s and achieved HBM GB/s (% of B200 peak), 1 GPU"
 UNIT = "Gparams/s"
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SRC = os.path.join(ROOT, "mixed_precision_zero_b200", "csrc", "neox_shard.cu")
+KERNEL_SRCS = [os.path.join(ROOT, "mixed_precision_zero_b200", "csrc", f) for f in ("neox_shard.cu", "neox_common.cuh")]
 
 
 def log(*a):
@@ -75,8 +75,12 @@ def hbm_peak():
 
 
 def kernel_source_hash() -> str:
-    with open(KERNEL_SRC, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Hash of the sources of the flat-shard kernels (the ones bench.py times)."""
+    h = hashlib.sha256()
+    for path in KERNEL_SRCS:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def recorded_traffic(workload: str):
