@@ -9,7 +9,9 @@ overflow flag, global norm, loss scaler, clip coefficient) and pass 2 (AdamW on
 FP32 master/m/v + cast to the 16-bit working copy).  Inputs are resident in HBM
 (22.6 GB for the default 1.41e9-parameter shard, far above the 126 MB L2, so no
 flush is needed between steps).  Under torchrun every rank steps its own shard of
-the same size (weak scaling); the per-rank step has no data-path collective.
+the same size (weak scaling) with the split step: pass 1, a 16-byte NCCL
+all-reduce of {sum of squares, non-finite flag}, then the shared decision and
+pass 2, as data-parallel ranks with one global norm and loss scale do.
 
 Prints one JSON line (rank 0).
 """
@@ -46,6 +48,8 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["b200", "reference"], default="b200")
     p.add_argument("--workload", default="pythia_1p4b")
     p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--split", action="store_true",
+                   help="run the split step (statistics, all-reduce, apply) even on one rank")
     p.add_argument("--api", choices=["flat", "multi"], default="flat",
                    help="flat: neox_shard_step; multi: neox_multi_step with one tensor per segment")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline")
@@ -378,7 +382,7 @@ def run_b200(args):
         log(f"note: --gpus {args.gpus} but WORLD_SIZE {ws}; using WORLD_SIZE")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if ws > 1:
+    if ws > 1 or (args.split and "RANK" in os.environ):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
     wl = W.ALL[args.workload]()
@@ -387,8 +391,23 @@ def run_b200(args):
     p1b, p2b = alg_bytes_per_param(wl.K, acc)
     stream = torch.cuda.current_stream()
 
+    # One step.  A single GPU runs the fused step; several ranks run the split
+    # step, all-reducing the 16 bytes of pass-1 statistics (NCCL) so that every
+    # rank takes the same overflow / scale / clip decision.
+    stats = torch.zeros(2, dtype=torch.float64, device=dev)
+
+    split = ws > 1 or args.split
+
+    def one_step():
+        if not split:
+            return shard.step(grads, params, wl.lr)
+        shard.grad_stats(grads, params, stats)
+        if dist.is_initialized():
+            dist.all_reduce(stats)
+        return shard.apply(grads, params, wl.lr, stats)
+
     for _ in range(args.warmup):
-        res = shard.step(grads, params, wl.lr)
+        res = one_step()
     t_before = shard.get_state()[2]
     shard.reset_profile()
     shard.set_profiling(True)
@@ -400,7 +419,7 @@ def run_b200(args):
     with ClockSampler(local) as clocks:
         ev0.record(stream)
         for _ in range(args.steps):
-            res = shard.step(grads, params, wl.lr)
+            res = one_step()
         ev1.record(stream)
         torch.cuda.synchronize()
     if ws > 1:
@@ -416,7 +435,7 @@ def run_b200(args):
     total_params = sum_over_ranks(float(wl.numel), dev)
     ms_step = ms / args.steps
     value = total_params * args.steps / (ms * 1e-3) / 1e9
-    p1_ms = prof.grad_pass_ms / prof.steps
+    p1_ms = prof.grad_pass_ms / prof.steps if not split else None  # split steps time only the decision there
     p2_ms = prof.update_pass_ms / prof.steps
     peak, peak_kind = hbm_peak()
     achieved = p2b * wl.numel / (p2_ms * 1e-3) / 1e9
@@ -494,7 +513,8 @@ def run_b200(args):
                    "element_offset": wl.elem_offset, "loss_scale": wl.bench_scale or wl.init_scale,
                    "state": "fp32 master/m/v",
                    "l2": f"inputs {(14 + 2 * wl.K) * wl.numel / 1e9:.1f} GB per rank >> 126 MB L2; no flush",
-                   "parallelism": f"{ws} independent shard(s), one per GPU"},
+                   "parallelism": (f"dp{ws}: one shard per GPU, 16-byte NCCL all-reduce of the pass-1 statistics "
+                                   "per step" if split else "one shard on one GPU")},
         "hbm": {"step_gbs": step_gbs, "step_frac": step_gbs / peak, "bytes_per_param": p1b + p2b,
                 "peak_gbs": peak, "peak_kind": peak_kind},
         "roofline": {"bound": "hbm", "kernel": "adam_kernel (pass 2)", "achieved": achieved, "peak": peak,
@@ -511,7 +531,7 @@ def run_b200(args):
     if cpu:
         line["cpu_baseline"] = cpu
     shard.close()
-    if ws > 1:
+    if dist.is_initialized():
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:

@@ -168,6 +168,32 @@ neox_status neox_shard_step(neox_shard* h, const void* const* grads, int32_t num
 neox_status neox_shard_step_async(neox_shard* h, const void* const* grads, int32_t num_grads, void* params,
                                   float lr, const float* lr_device, void* cuda_stream, neox_step_result* result);
 
+/* The step split around the one exchange data-parallel ranks need.
+ *
+ * With ZeRO stage 1/2 every rank owns one shard ("GPT-NeoX: how it opened the
+ * door to democratised 100B-scale training" (ainews.cool), "技术深度解析"),
+ * but the overflow flag and the global gradient norm -- hence the loss-scale
+ * trajectory and the clip coefficient -- are properties of the whole model.
+ * Each rank therefore runs:
+ *   1. neox_shard_grad_stats: pass 1 over its shard; writes two doubles to
+ *      stats_device: [0] = sum of squares of its unscaled gradients,
+ *      [1] = 1.0 if any of them is not finite, else 0.0;
+ *   2. an all-reduce (SUM) of those 16 bytes across the ranks, by the caller
+ *      (e.g. NCCL through torch.distributed), on the same stream;
+ *   3. neox_shard_apply: one single-thread kernel takes the step's decisions
+ *      (overflow = [1] > 0, norm = sqrt([0]), scaler, clip coefficient, t)
+ *      from the reduced statistics, then pass 2 updates the shard; it waits
+ *      for the step and fills `out` like neox_shard_step.
+ * Every rank then holds the same scale, counters and clip coefficient.  The
+ * grads, num_grads and params of both calls must be the same (pass 2 re-reads
+ * the gradients; params fixes the vector layout); stats_device is 8-byte
+ * aligned device memory the caller owns.  With one rank (no all-reduce) the
+ * two calls give exactly the result of neox_shard_step. */
+neox_status neox_shard_grad_stats(neox_shard* h, const void* const* grads, int32_t num_grads, void* params,
+                                  void* cuda_stream, double* stats_device);
+neox_status neox_shard_apply(neox_shard* h, const void* const* grads, int32_t num_grads, void* params, float lr,
+                             const double* stats_device, void* cuda_stream, neox_step_result* out);
+
 /* Replace the hyperparameters (e.g. the clip 1.0 -> 0.3 change); the current
  * loss scale and counters are kept (init_scale is ignored here). */
 neox_status neox_shard_set_hparams(neox_shard* h, const neox_hparams* hp);

@@ -24,7 +24,7 @@ from ._abi import (NEOX_BF16, NEOX_ERR_CUDA, NEOX_ERR_INVALID_ARGUMENT, NEOX_ERR
                    neox_shard_step, neox_shard_step_async, neox_status_string, neox_step_result,
                    neox_tensor, neox_tensor_set, neox_multi_create, neox_multi_step, neox_multi_step_async,
                    neox_multi_rebind_grads, neox_multi_get_state, neox_multi_set_state,
-                   neox_multi_set_hparams, neox_multi_destroy)
+                   neox_multi_set_hparams, neox_multi_destroy, neox_shard_grad_stats, neox_shard_apply)
 
 __all__ = ["NeoxShard", "NeoxMultiShard", "Hparams", "NeoxError", "neox_shard_create", "neox_shard_step",
            "neox_shard_destroy", "neox_shard_set_hparams", "neox_shard_get_state",
@@ -115,6 +115,28 @@ class NeoxShard:
         neox_shard_step_async(self.handle, [g.data_ptr() for g in grads], params.data_ptr(), lr, sp,
                               None if result is None else result.data_ptr(),
                               None if lr_device is None else lr_device.data_ptr())
+
+    def grad_stats(self, grads, params, stats, stream=None) -> None:
+        """Pass 1 only: `stats` (float64 CUDA tensor of 2) receives this shard's
+        {sum of squares, non-finite flag}; all-reduce it (SUM) across ranks,
+        then call apply()."""
+        import torch
+        self._check(grads, params)
+        if stats.dtype != torch.float64 or stats.numel() < 2 or not stats.is_cuda:
+            raise ValueError("stats must be a float64 CUDA tensor of 2 elements")
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device)
+        sp = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+        neox_shard_grad_stats(self.handle, [g.data_ptr() for g in grads], params.data_ptr(), sp, stats.data_ptr())
+
+    def apply(self, grads, params, lr: float, stats, stream=None) -> neox_step_result:
+        """The step's decisions from the (all-reduced) statistics, then pass 2."""
+        import torch
+        self._check(grads, params)
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device)
+        sp = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+        return neox_shard_apply(self.handle, [g.data_ptr() for g in grads], params.data_ptr(), lr, stats.data_ptr(), sp)
 
     def set_hparams(self, hp: Hparams) -> None:
         neox_shard_set_hparams(self.handle, hp.c())

@@ -92,6 +92,13 @@ def lib() -> ctypes.CDLL:
         L.neox_shard_step_async.argtypes = [_H, ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32, ctypes.c_void_p,
                                             ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
         L.neox_shard_step_async.restype = S
+        L.neox_shard_grad_stats.argtypes = [_H, ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32, ctypes.c_void_p,
+                                            ctypes.c_void_p, ctypes.c_void_p]
+        L.neox_shard_grad_stats.restype = S
+        L.neox_shard_apply.argtypes = [_H, ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32, ctypes.c_void_p,
+                                       ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
+                                       ctypes.POINTER(neox_step_result)]
+        L.neox_shard_apply.restype = S
         L.neox_shard_set_hparams.argtypes = [_H, ctypes.POINTER(neox_hparams)]
         L.neox_shard_set_hparams.restype = S
         L.neox_shard_get_state.argtypes = [_H, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int32),
@@ -177,6 +184,22 @@ def neox_shard_step_async(h: int, grad_ptrs, params_ptr: int, lr: float, stream:
     st = lib().neox_shard_step_async(h, arr, len(grad_ptrs), params_ptr, lr, lr_device_ptr, stream, result_ptr)
     if st != NEOX_OK:
         raise NeoxError(st, lib().neox_last_error(h).decode())
+
+
+def neox_shard_grad_stats(h: int, grad_ptrs, params_ptr: int, stream: int, stats_ptr: int) -> None:
+    arr = (ctypes.c_void_p * len(grad_ptrs))(*grad_ptrs)
+    st = lib().neox_shard_grad_stats(h, arr, len(grad_ptrs), params_ptr, stream, stats_ptr)
+    if st != NEOX_OK:
+        raise NeoxError(st, lib().neox_last_error(h).decode())
+
+
+def neox_shard_apply(h: int, grad_ptrs, params_ptr: int, lr: float, stats_ptr: int, stream: int) -> neox_step_result:
+    arr = (ctypes.c_void_p * len(grad_ptrs))(*grad_ptrs)
+    res = neox_step_result()
+    st = lib().neox_shard_apply(h, arr, len(grad_ptrs), params_ptr, lr, stats_ptr, stream, ctypes.byref(res))
+    if st != NEOX_OK:
+        raise NeoxError(st, lib().neox_last_error(h).decode())
+    return res
 
 
 def neox_shard_set_hparams(h: int, hp: neox_hparams) -> None:

@@ -71,6 +71,9 @@ struct ScalerArgs {
     float lr, beta1, beta2;
     const float* lr_ptr;       // when non-NULL, the learning rate is read here
     neox_step_result* result;  // device-accessible; NULL = not written
+    // split step: pass 1 writes {sum of squares, non-finite flag} here and
+    // takes no decision (the ranks' statistics are all-reduced first)
+    double* stats_out;
 };
 
 struct AdamArgs {
@@ -320,40 +323,11 @@ __device__ __forceinline__ void block_reduce(double& s, int& bad, double* sh_s, 
 // loss scaler, clip coefficient, applied-step count; for asynchronous steps
 // also the bias corrections and the caller's result record).  No spinning:
 // every block but the last simply returns.
-template <int THREADS>
-__device__ __forceinline__ void finish_pass1(double s, int bad, double* __restrict__ part_s, int* __restrict__ part_b,
-                                             DevScalars* __restrict__ sc, const ScalerArgs& sa, double* sh_s, int* sh_b,
-                                             bool* is_last_sh) {
-    bool& is_last = *is_last_sh;
-    // Let the update kernel's blocks start their prologue as this grid winds
-    // down; they wait (griddepcontrol.wait) for this grid's completion before
-    // reading anything it writes.
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    block_reduce<THREADS>(s, bad, sh_s, sh_b);
-    if (threadIdx.x == 0) {
-        part_s[blockIdx.x] = s;
-        part_b[blockIdx.x] = bad;
-        __threadfence();
-        const unsigned ticket = atomicAdd(&sc->blocks_done, 1u);
-        is_last = (ticket == gridDim.x - 1);
-    }
-    __syncthreads();
-    if (!is_last) return;
-
-    // Last block: every other block's partial is visible (each fenced before
-    // taking its ticket).  Reduce them in a fixed order.
-    __threadfence();
-    s = 0.0;
-    bad = 0;
-    for (unsigned j = threadIdx.x; j < gridDim.x; j += THREADS) {
-        s += __ldcg(part_s + j);
-        bad |= __ldcg(part_b + j);
-    }
-    __syncthreads();
-    block_reduce<THREADS>(s, bad, sh_s, sh_b);
-    if (threadIdx.x != 0) return;
-
-    // Scalar decisions of the step.
+// The scalar decisions of a step from its global sum of squares `s` and
+// non-finite flag `bad`: overflow, norm, dynamic loss scaler, clip
+// coefficient, applied-step count; for asynchronous steps also the bias
+// corrections and the caller's result record.  One thread.
+__device__ __forceinline__ void decide_step(DevScalars* __restrict__ sc, const ScalerArgs& sa, double s, int bad) {
     int overflow = bad != 0;
     const double norm = sqrt(s);
     if (!overflow && !isfinite(norm)) overflow = 1;
@@ -408,6 +382,47 @@ __device__ __forceinline__ void finish_pass1(double s, int bad, double* __restri
             r->applied_steps = t;
         }
     }
+}
+
+template <int THREADS>
+__device__ __forceinline__ void finish_pass1(double s, int bad, double* __restrict__ part_s, int* __restrict__ part_b,
+                                             DevScalars* __restrict__ sc, const ScalerArgs& sa, double* sh_s, int* sh_b,
+                                             bool* is_last_sh) {
+    bool& is_last = *is_last_sh;
+    // Let the update kernel's blocks start their prologue as this grid winds
+    // down; they wait (griddepcontrol.wait) for this grid's completion before
+    // reading anything it writes.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    block_reduce<THREADS>(s, bad, sh_s, sh_b);
+    if (threadIdx.x == 0) {
+        part_s[blockIdx.x] = s;
+        part_b[blockIdx.x] = bad;
+        __threadfence();
+        const unsigned ticket = atomicAdd(&sc->blocks_done, 1u);
+        is_last = (ticket == gridDim.x - 1);
+    }
+    __syncthreads();
+    if (!is_last) return;
+
+    // Last block: every other block's partial is visible (each fenced before
+    // taking its ticket).  Reduce them in a fixed order.
+    __threadfence();
+    s = 0.0;
+    bad = 0;
+    for (unsigned j = threadIdx.x; j < gridDim.x; j += THREADS) {
+        s += __ldcg(part_s + j);
+        bad |= __ldcg(part_b + j);
+    }
+    __syncthreads();
+    block_reduce<THREADS>(s, bad, sh_s, sh_b);
+    if (threadIdx.x != 0) return;
+
+    if (sa.stats_out) {  // split step: publish the statistics, decide later
+        sa.stats_out[0] = s;
+        sa.stats_out[1] = bad ? 1.0 : 0.0;
+    } else {
+        decide_step(sc, sa, s, bad);
+    }
     sc->blocks_done = 0;
 }
 
@@ -428,6 +443,12 @@ __device__ __forceinline__ void adam_vec(const float (&g)[VEC], const float (&ke
         v[e] = vj;
         p[e] = pj;
     }
+}
+
+// The decision of a split step from all-reduced statistics {sum of squares,
+// number of ranks that saw a non-finite value}.  One thread.
+__global__ void decide_kernel(DevScalars* __restrict__ sc, ScalerArgs sa, const double* __restrict__ stats) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) decide_step(sc, sa, stats[0], stats[1] != 0.0);
 }
 
 // ---------------------------------------------------------------- host helpers

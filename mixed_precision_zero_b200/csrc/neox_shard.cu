@@ -402,9 +402,11 @@ neox_status refresh_mirror(neox_shard* h) {
 // steps, whose caller keeps that copy current).  device_bc = true: the last
 // pass-1 block forms them from the device step count and writes `result`.
 // timed: record the profiling events around the two launches.
+enum StepMode { kFused = 0, kStatsOnly = 1, kApply = 2 };
+
 neox_status enqueue_step(neox_shard* h, const void* const* grads, int32_t num_grads, void* params, float lr,
                          const float* lr_dev, cudaStream_t st, bool device_bc, neox_step_result* result,
-                         bool timed) {
+                         bool timed, StepMode mode = kFused, double* stats = nullptr) {
     if (num_grads < 1 || num_grads > kMaxGrads) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "num_grads must be in [1, 64]");
     if (!grads) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "grads is NULL");
     if (!lr_dev && (!finite(lr) || lr < 0.0f)) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "lr must be finite and >= 0");
@@ -423,6 +425,8 @@ neox_status enqueue_step(neox_shard* h, const void* const* grads, int32_t num_gr
         a16[num_grads] = (uintptr_t)params;
     }
     if (result && ((uintptr_t)result & 7u)) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "result must be 8-byte aligned");
+    if (mode != kFused && (!stats || ((uintptr_t)stats & 7u)))
+        return fail(h, NEOX_ERR_INVALID_ARGUMENT, "stats must be a non-NULL, 8-byte aligned device pointer");
     if (lr_dev && ((uintptr_t)lr_dev & 3u)) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "lr_device must be 4-byte aligned");
 
     const bool use_acc = num_grads >= 5 && h->d_acc != nullptr;
@@ -448,6 +452,7 @@ neox_status enqueue_step(neox_shard* h, const void* const* grads, int32_t num_gr
     sa.beta2 = h->hp.beta2;
     sa.lr_ptr = lr_dev;
     sa.result = result;
+    sa.stats_out = mode == kStatsOnly ? stats : nullptr;
 
     AdamArgs a{};
     a.lr = lr;
@@ -469,12 +474,17 @@ neox_status enqueue_step(neox_shard* h, const void* const* grads, int32_t num_gr
 
     cudaError_t e;
     if (timed && (e = cudaEventRecord(h->ev[0], st)) != cudaSuccess) return cuda_fail(h, e, "cudaEventRecord");
-    if (h->gdtype == NEOX_FP16) e = dispatch1v<F16>(h, vec, gp, num_grads, L, sa, acc, st);
-    else e = dispatch1v<BF16>(h, vec, gp, num_grads, L, sa, acc, st);
-    if (e != cudaSuccess) return cuda_fail(h, e, "pass-1 launch");
+    if (mode == kApply) {  // the decision from the all-reduced statistics
+        decide_kernel<<<1, 1, 0, st>>>(h->d_sc, sa, stats);
+        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(h, e, "decision launch");
+    } else {
+        if (h->gdtype == NEOX_FP16) e = dispatch1v<F16>(h, vec, gp, num_grads, L, sa, acc, st);
+        else e = dispatch1v<BF16>(h, vec, gp, num_grads, L, sa, acc, st);
+        if (e != cudaSuccess) return cuda_fail(h, e, "pass-1 launch");
+    }
     h->prof.launches += 1;
     if (timed && (e = cudaEventRecord(h->ev[1], st)) != cudaSuccess) return cuda_fail(h, e, "cudaEventRecord");
-    if (h->numel > 0) {
+    if (h->numel > 0 && mode != kStatsOnly) {
         uint16_t* w = static_cast<uint16_t*>(params);
         if (h->gdtype == NEOX_FP16) {
             e = h->wdtype == NEOX_FP16 ? dispatch2v<F16, F16>(h, vec, gp, num_grads, acc, L, a, w, st)
@@ -487,6 +497,37 @@ neox_status enqueue_step(neox_shard* h, const void* const* grads, int32_t num_gr
         h->prof.launches += 1;
     }
     if (timed && (e = cudaEventRecord(h->ev[2], st)) != cudaSuccess) return cuda_fail(h, e, "cudaEventRecord");
+    return NEOX_OK;
+}
+
+// Wait for the step on `st`, read its scalar block, fill `out`, refresh the
+// host copy of the scaler state and account the profiling events.
+neox_status read_result(neox_shard* h, cudaStream_t st, neox_step_result* out) {
+    cudaError_t e;
+    if ((e = cudaMemcpyAsync(h->h_sc, h->d_sc, sizeof(DevScalars), cudaMemcpyDeviceToHost, st)) != cudaSuccess)
+        return cuda_fail(h, e, "cudaMemcpyAsync result");
+    if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(h, e, "step execution");
+    const DevScalars& r = *h->h_sc;
+    out->overflow = r.overflow;
+    out->grad_norm = r.norm;
+    out->clip_coef = r.coef;
+    out->loss_scale = r.scale_used;
+    out->loss_scale_next = r.scale;
+    out->good_steps = r.good;
+    out->applied_steps = r.t;
+    h->scale = r.scale;
+    h->good = r.good;
+    h->t = r.t;
+    if (h->profiling) {
+        float t01 = 0.f, t12 = 0.f;
+        cudaEventElapsedTime(&t01, h->ev[0], h->ev[1]);
+        cudaEventElapsedTime(&t12, h->ev[1], h->ev[2]);
+        h->prof.steps += 1;
+        h->prof.grad_pass_ms += t01;
+        h->prof.update_pass_ms += t12;
+        h->prof.last_grad_pass_ms = t01;
+        h->prof.last_update_pass_ms = t12;
+    }
     return NEOX_OK;
 }
 
@@ -712,34 +753,7 @@ neox_status neox_shard_step(neox_shard* h, const void* const* grads, int32_t num
                                      h->profiling);
         s != NEOX_OK)
         return s;
-    cudaError_t e;
-    if ((e = cudaMemcpyAsync(h->h_sc, h->d_sc, sizeof(DevScalars), cudaMemcpyDeviceToHost, st)) != cudaSuccess)
-        return cuda_fail(h, e, "cudaMemcpyAsync result");
-    if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(h, e, "step execution");
-
-    const DevScalars& r = *h->h_sc;
-    out->overflow = r.overflow;
-    out->grad_norm = r.norm;
-    out->clip_coef = r.coef;
-    out->loss_scale = r.scale_used;
-    out->loss_scale_next = r.scale;
-    out->good_steps = r.good;
-    out->applied_steps = r.t;
-    h->scale = r.scale;
-    h->good = r.good;
-    h->t = r.t;
-
-    if (h->profiling) {
-        float t01 = 0.f, t12 = 0.f;
-        cudaEventElapsedTime(&t01, h->ev[0], h->ev[1]);
-        cudaEventElapsedTime(&t12, h->ev[1], h->ev[2]);
-        h->prof.steps += 1;
-        h->prof.grad_pass_ms += t01;
-        h->prof.update_pass_ms += t12;
-        h->prof.last_grad_pass_ms = t01;
-        h->prof.last_update_pass_ms = t12;
-    }
-    return NEOX_OK;
+    return read_result(h, st, out);
 }
 
 neox_status neox_shard_step_async(neox_shard* h, const void* const* grads, int32_t num_grads, void* params,
@@ -751,6 +765,31 @@ neox_status neox_shard_step_async(neox_shard* h, const void* const* grads, int32
     if (!g.ok) return fail(h, NEOX_ERR_CUDA, "cudaSetDevice failed");
     h->async_used = true;
     return enqueue_step(h, grads, num_grads, params, lr, lr_device, st, true, result, false);
+}
+
+neox_status neox_shard_grad_stats(neox_shard* h, const void* const* grads, int32_t num_grads, void* params,
+                                  void* cuda_stream, double* stats_device) {
+    if (!h) return NEOX_ERR_INVALID_ARGUMENT;
+    h->last_error.clear();
+    DeviceGuard g(h->device);
+    if (!g.ok) return fail(h, NEOX_ERR_CUDA, "cudaSetDevice failed");
+    return enqueue_step(h, grads, num_grads, params, 0.0f, nullptr, static_cast<cudaStream_t>(cuda_stream), false,
+                        nullptr, false, kStatsOnly, stats_device);
+}
+
+neox_status neox_shard_apply(neox_shard* h, const void* const* grads, int32_t num_grads, void* params, float lr,
+                             const double* stats_device, void* cuda_stream, neox_step_result* out) {
+    if (!h) return NEOX_ERR_INVALID_ARGUMENT;
+    h->last_error.clear();
+    if (!out) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "out is NULL");
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    DeviceGuard g(h->device);
+    if (!g.ok) return fail(h, NEOX_ERR_CUDA, "cudaSetDevice failed");
+    if (neox_status s = enqueue_step(h, grads, num_grads, params, lr, nullptr, st, h->async_used, nullptr,
+                                     h->profiling, kApply, const_cast<double*>(stats_device));
+        s != NEOX_OK)
+        return s;
+    return read_result(h, st, out);
 }
 
 }  // extern "C"
