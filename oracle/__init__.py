@@ -47,11 +47,12 @@ class Hparams(ctypes.Structure):
     _fields_ = [("beta1", ctypes.c_float), ("beta2", ctypes.c_float), ("eps", ctypes.c_float),
                 ("clip_norm", ctypes.c_float), ("predivide", ctypes.c_float),
                 ("scale_factor", ctypes.c_float), ("min_scale", ctypes.c_float),
-                ("scale_window", ctypes.c_int32)]
+                ("scale_window", ctypes.c_int32), ("hysteresis", ctypes.c_int32), ("optimizer", ctypes.c_int32)]
 
 
 class Scaler(ctypes.Structure):
-    _fields_ = [("scale", ctypes.c_float), ("good", ctypes.c_int32), ("t", ctypes.c_int64)]
+    _fields_ = [("scale", ctypes.c_float), ("good", ctypes.c_int32), ("t", ctypes.c_int64),
+                ("hyst", ctypes.c_int32), ("pad_", ctypes.c_int32)]
 
 
 class Segment(ctypes.Structure):
@@ -117,6 +118,9 @@ def _configure(L):
     L.orc_adam_apply.argtypes = [_U64, _P, _U64, _P, ctypes.c_int32, ctypes.c_int32,
                                  _P, ctypes.c_int32, _P, _P, _P, _P, ctypes.c_int32,
                                  ctypes.POINTER(Hparams), ctypes.c_float, ctypes.POINTER(StepInfo)]
+    L.orc_sgd_apply.argtypes = [_U64, _P, _U64, _P, ctypes.c_int32, ctypes.c_int32, _P, ctypes.c_int32,
+                                _P, _P, ctypes.c_int32, ctypes.POINTER(Hparams), ctypes.c_float,
+                                ctypes.POINTER(StepInfo)]
     L.orc_step_decide.argtypes = [ctypes.POINTER(Hparams), ctypes.POINTER(Scaler), ctypes.c_float,
                                   ctypes.c_int64, ctypes.c_double, ctypes.POINTER(StepInfo)]
     L.orc_step.argtypes = [_U64, _P, ctypes.c_int32, ctypes.c_int32, _P, ctypes.c_int32,
@@ -201,10 +205,16 @@ class OracleHparams:
     scale_factor: float = 2.0
     min_scale: float = 1.0
     scale_window: int = 1000
+    hysteresis: int = 1
+    optimizer: int = 0          # 0 AdamW, 1 SGD
 
     def c(self) -> Hparams:
         return Hparams(self.beta1, self.beta2, self.eps, self.clip_norm, self.predivide,
-                       self.scale_factor, self.min_scale, self.scale_window)
+                       self.scale_factor, self.min_scale, self.scale_window, self.hysteresis, self.optimizer)
+
+    @property
+    def hyst0(self) -> int:
+        return max(1, self.hysteresis)
 
 
 def segments_array(segments, n: int, default_wd: float):
@@ -215,9 +225,14 @@ def segments_array(segments, n: int, default_wd: float):
     return arr
 
 
-def scaler_update(hp: OracleHparams, scale: float, good: int, t: int, overflow: bool):
-    sc = Scaler(scale, good, t)
+def scaler_update(hp: OracleHparams, scale: float, good: int, t: int, overflow: bool, hyst: int | None = None,
+                  with_hyst: bool = False):
+    """One scaler update; `hyst` is the hysteresis count (None: a full one,
+    which is exact whenever hysteresis <= 1)."""
+    sc = Scaler(scale, good, t, hp.hyst0 if hyst is None else hyst, 0)
     lib().orc_scaler_update(ctypes.byref(hp.c()), ctypes.byref(sc), int(overflow))
+    if with_hyst:
+        return sc.scale, sc.good, sc.t, sc.hyst
     return sc.scale, sc.good, sc.t
 
 
@@ -275,6 +290,15 @@ def adam_apply(index, first: int, grads, gbf16: bool, segs, master, m, v, w, wbf
                          ctypes.byref(hp.c()), lr, ctypes.byref(info))
 
 
+def sgd_apply(index, first: int, grads, gbf16: bool, segs, master, w, wbf16: bool, hp: OracleHparams, lr: float,
+              info: StepInfo):
+    """SGD update of the elements whose gradients are `grads` (see adam_apply)."""
+    n = master.size
+    idx_ptr = None if index is None else _ptr(np.ascontiguousarray(index, dtype=np.uint64))
+    lib().orc_sgd_apply(n, idx_ptr, first, _grad_ptrs(grads), len(grads), int(gbf16), segs, len(segs), _ptr(master),
+                        _ptr(w), int(wbf16), ctypes.byref(hp.c()), lr, ctypes.byref(info))
+
+
 @dataclass
 class OracleShard:
     """A whole shard held in host memory, stepped by the single-threaded oracle."""
@@ -292,7 +316,7 @@ class OracleShard:
         self.v = np.zeros(n, np.float32)
         self.w = encode16(self.master, self.wbf16)
         self.segs = segments_array(self.segments, n, self.default_wd)
-        self.scaler = Scaler(self.hp.init_scale, 0, 0)
+        self.scaler = Scaler(self.hp.init_scale, 0, 0, self.hp.hyst0, 0)
 
     @property
     def scale(self) -> float:
@@ -324,7 +348,7 @@ class Oracle64Shard:
         self.m = np.zeros(n, np.float64)
         self.v = np.zeros(n, np.float64)
         self.segs = segments_array(self.segments, n, self.default_wd)
-        self.scaler = Scaler(self.hp.init_scale, 0, 0)
+        self.scaler = Scaler(self.hp.init_scale, 0, 0, self.hp.hyst0, 0)
 
     def step(self, grads, lr: float):
         grads = [np.ascontiguousarray(g, dtype=np.uint16) for g in grads]

@@ -36,7 +36,10 @@
  *  - overflow = any non-finite unscaled gradient element, or a non-finite norm;
  *  - on overflow the step is skipped: no state changes, the applied-step count
  *    t does not advance, the scale drops by scale_factor (floored at min_scale)
- *    and the growth counter resets;
+ *    and the growth counter resets; with a hysteresis h > 1 the scale drops
+ *    only once h overflows happened since the last growth (Megatron-style);
+ *  - the SGD fallback is plain SGD without momentum, with the same decoupled
+ *    weight decay as AdamW;
  *  - after scale_window consecutive applied steps the scale grows by
  *    scale_factor (unless the grown scale would not be finite) and the
  *    counter resets;
@@ -154,12 +157,17 @@ typedef struct {
     float scale_factor;   /* loss-scale growth / backoff factor       [OPT-CS] */
     float min_scale;      /* floor of the loss scale                  [OPT-BN] */
     int32_t scale_window; /* applied steps between scale growths               */
+    int32_t hysteresis;   /* overflows since the last growth before a back-off
+                             (<= 1: back off at every overflow)                */
+    int32_t optimizer;    /* 0: AdamW; 1: SGD, the fallback tried   [OPT-MA] */
 } orc_hparams;
 
 typedef struct {
     float scale;          /* S: the loss scale the current grads carry */
     int32_t good;         /* consecutive applied steps since the last change */
     int64_t t;            /* applied (non-skipped) Adam steps */
+    int32_t hyst;         /* overflows still tolerated before a back-off */
+    int32_t pad_;
 } orc_scaler;
 
 typedef struct {
@@ -233,15 +241,23 @@ void orc_grad_stats(const uint16_t* const* g, int32_t K, int32_t gbf16, uint64_t
 }
 
 /* Dynamic loss scaler.                                  [OPT-CS][OPT-BN][OPT-MA]
- * overflow: S <- max(S / factor, min_scale), counter reset, step skipped.
+ * overflow: step skipped, counter reset; the hysteresis count drops by one
+ *           (not below 0) and, once it is 0, S <- max(S / factor, min_scale).
+ *           With hysteresis <= 1 that is every overflow.
  * applied:  counter + 1; at scale_window: S <- S * factor unless that is not
- *           finite (then S stays), counter reset. */
+ *           finite (then S stays), counter reset, hysteresis count refilled. */
+int32_t orc_hysteresis(const orc_hparams* hp) { return hp->hysteresis > 1 ? hp->hysteresis : 1; }
+
 void orc_scaler_update(const orc_hparams* hp, orc_scaler* sc, int32_t overflow)
 {
     if (overflow) {
-        float s = sc->scale / hp->scale_factor;
-        sc->scale = s > hp->min_scale ? s : hp->min_scale;
         sc->good = 0;
+        if (sc->hyst > 0)
+            sc->hyst -= 1;
+        if (sc->hyst == 0) {
+            float s = sc->scale / hp->scale_factor;
+            sc->scale = s > hp->min_scale ? s : hp->min_scale;
+        }
         return;
     }
     sc->good += 1;
@@ -250,6 +266,7 @@ void orc_scaler_update(const orc_hparams* hp, orc_scaler* sc, int32_t overflow)
         if (isfinite(s))            /* a scale never grows to infinity */
             sc->scale = s;
         sc->good = 0;
+        sc->hyst = orc_hysteresis(hp);
     }
 }
 
@@ -317,6 +334,34 @@ void orc_adam_apply(uint64_t n, const uint64_t* index, uint64_t first,
     }
 }
 
+/* Plain SGD (no momentum) with the same decoupled weight decay, the
+ * alternative optimizer the OPT run tried:                           [OPT-MA]
+ * p <- p(1 - lr*wd) - lr * (g*c); the moments are left untouched. */
+void orc_sgd_apply(uint64_t n, const uint64_t* index, uint64_t first,
+                   const uint16_t* const* g, int32_t K, int32_t gbf16,
+                   const orc_segment* segs, int32_t nsegs,
+                   float* master, uint16_t* w, int32_t wbf16,
+                   const orc_hparams* hp, float lr, const orc_step_info* info)
+{
+    float inv_pre, inv_us;
+    orc_ingest_factors(K, hp->predivide, info->scale_used, &inv_pre, &inv_us);
+    const float c = info->coef;
+    for (uint64_t j = 0; j < n; j++) {
+        uint64_t idx = index ? index[j] : first + j;
+        float wd = segment_wd(segs, nsegs, idx);
+        float gj = unscaled_grad(g, K, gbf16, j, inv_pre, inv_us);
+        float g_clipped = gj * c;
+        float q = master[j];
+        float lr_wd = lr * wd;
+        float retain = 1.0f - lr_wd;     /* decoupled decay */
+        q = q * retain;
+        float delta = lr * g_clipped;    /* gradient step   */
+        q = q - delta;
+        master[j] = q;
+        w[j] = enc16(q, wbf16);
+    }
+}
+
 /* The per-step scalar decisions, given the pass-1 results: overflow, norm,
  * scaler, clip coefficient, applied-step count and bias corrections.
  * Returns the info the update needs; updates the scaler state in place. */
@@ -363,9 +408,13 @@ int32_t orc_step(uint64_t n, const uint16_t* const* g, int32_t K, int32_t gbf16,
     double sumsq;
     orc_grad_stats(g, K, gbf16, n, inv_pre, inv_us, &bad, &sumsq);
     orc_step_decide(hp, sc, lr, bad, sumsq, info);
-    if (!info->overflow)
-        orc_adam_apply(n, NULL, 0, g, K, gbf16, segs, nsegs,
-                       master, m, v, w, wbf16, hp, lr, info);
+    if (!info->overflow) {
+        if (hp->optimizer == 1)
+            orc_sgd_apply(n, NULL, 0, g, K, gbf16, segs, nsegs, master, w, wbf16, hp, lr, info);
+        else
+            orc_adam_apply(n, NULL, 0, g, K, gbf16, segs, nsegs,
+                           master, m, v, w, wbf16, hp, lr, info);
+    }
     return info->overflow;
 }
 
@@ -415,6 +464,11 @@ int32_t orc64_step(uint64_t n, const uint16_t* const* g, int32_t K, int32_t gbf1
         for (int32_t k = 0; k < K; k++)
             a += (double)dec16(g[k][j], gbf16) / (double)hp->predivide;
         double gh = a / (post * S) * c;
+        if (hp->optimizer == 1) {  /* SGD */
+            double wd = segment_wd(segs, nsegs, j);
+            master[j] = master[j] * (1.0 - lrd * wd) - lrd * gh;
+            continue;
+        }
         m[j] = b1 * m[j] + (1.0 - b1) * gh;
         v[j] = b2 * v[j] + (1.0 - b2) * gh * gh;
         double wd = segment_wd(segs, nsegs, j);

@@ -40,10 +40,11 @@ MUTANTS = [
     ("norm not rooted", "    double norm = sqrt(sumsq);\n    if (!overflow", "    double norm = sumsq;\n    if (!overflow"),
     ("clip margin dropped", "double c = (double)clip / (norm + 1e-6);", "double c = (double)clip / norm;"),
     ("inf not detected", "        if (!isfinite(x))\n            bad++;", "        if (isnan(x))\n            bad++;"),
-    ("overflow applies update", "    if (!info->overflow)\n        orc_adam_apply", "    if (1)\n        orc_adam_apply"),
+    ("overflow applies update", "    if (!info->overflow) {\n        if (hp->optimizer == 1)",
+     "    if (1) {\n        if (hp->optimizer == 1)"),
     ("overflow advances t", "        info->coef = 0.0f;\n        info->t = sc->t;", "        info->coef = 0.0f;\n        sc->t += 1;\n        info->t = sc->t;"),
     ("backoff grows", "float s = sc->scale / hp->scale_factor;", "float s = sc->scale * hp->scale_factor;"),
-    ("counter kept on overflow", "        sc->good = 0;\n        return;", "        return;"),
+    ("counter kept on overflow", "    if (overflow) {\n        sc->good = 0;\n", "    if (overflow) {\n"),
     ("growth counter not reset", "            sc->scale = s;\n        sc->good = 0;", "            sc->scale = s;"),
     ("floor ignored", "sc->scale = s > hp->min_scale ? s : hp->min_scale;", "sc->scale = s;"),
     ("segment lookup off by one", "if (segs[mid].offset <= idx) lo = mid;", "if (segs[mid].offset < idx) lo = mid;"),
@@ -51,6 +52,11 @@ MUTANTS = [
     ("ties away from zero", "if (rem > half || (rem == half && (q & 1u)))", "if (rem >= half)"),
     ("f16 subnormal scale", "mag = ldexpf((float)frac, -24);", "mag = ldexpf((float)frac, -25);"),
     ("bf16 no rounding", "return (uint16_t)rne(x >> 16, x & 0xffffu, 0x8000u);", "return (uint16_t)(x >> 16);"),
+    ("hysteresis ignored", "        if (sc->hyst == 0) {", "        if (1) {"),
+    ("hysteresis never refilled", "        sc->hyst = orc_hysteresis(hp);", "        sc->hyst = 1;"),
+    ("sgd step sign", "        q = q - delta;", "        q = q + delta;"),
+    ("sgd ignores clip", "        float g_clipped = gj * c;", "        float g_clipped = gj;"),
+    ("sgd decay dropped", "        q = q * retain;", "        q = q * 1.0f;"),
 ]
 
 # pins run against each mutant, cheapest first
@@ -75,6 +81,9 @@ PINS = [
     (ts.test_scaler_matches_torch_gradscaler, {}),
     (ts.test_matches_torch_adamw_float64, {}),
     (ts.test_fp32_oracle_tracks_float64_brute_force, {"gbf16": False, "K": 3, "pre": 2.0}),
+    (ts.test_scaler_hysteresis_golden, {}),
+    (ts.test_sgd_matches_torch_float64, {}),
+    (ts.test_sgd_closed_form_and_untouched_moments, {}),
 ]
 
 

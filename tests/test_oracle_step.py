@@ -412,3 +412,76 @@ def test_state_accounting_oracle_arrays(orc):
     assert per == 16
     assert int(facts["params"]) * per == int(facts["state_bytes"])
     assert int(facts["params"]) * sh.w.itemsize == int(facts["fp16_weight_bytes"])
+
+
+# ---------------------------------------------------------------- scaler / optimizer variants
+
+def test_scaler_hysteresis_golden(orc):
+    facts = {}
+    for ln in open(os.path.join(GOLDEN, "scaler_hysteresis.txt")):
+        if ln.strip() and not ln.startswith("#"):
+            k, *v = ln.split()
+            facts[k] = [float(x) for x in v]
+    hp = orc.OracleHparams(init_scale=facts["init"][0], scale_factor=facts["factor"][0],
+                           scale_window=int(facts["window"][0]), hysteresis=int(facts["hysteresis"][0]))
+    ov = {int(x) for x in facts["overflows"]}
+    s, g, t, h = hp.init_scale, 0, 0, hp.hyst0
+    got = []
+    for call in range(1, len(facts["scales"]) + 1):
+        s, g, t, h = orc.scaler_update(hp, s, g, t, call in ov, hyst=h, with_hyst=True)
+        if call not in ov:
+            t += 1
+        got.append(s)
+    assert got == facts["scales"] and t == int(facts["applied"][0])
+    # hysteresis 0 or 1 is the plain scaler: a back-off at every overflow
+    # (same calls, worked by hand: 2, 3 halve; 6, 7, 8 halve; 11 grows; 12
+    # halves; 15 grows)
+    plain = [1024, 512, 256, 256, 256, 128, 64, 32, 32, 32, 64, 32, 32, 32, 64]
+    for h1 in (0, 1):
+        hp1 = orc.OracleHparams(init_scale=1024.0, scale_window=3, hysteresis=h1)
+        s, g, t, h = 1024.0, 0, 0, hp1.hyst0
+        got = []
+        for call in range(1, 16):
+            s, g, t, h = orc.scaler_update(hp1, s, g, t, call in ov, hyst=h, with_hyst=True)
+            got.append(s)
+        assert got == plain
+
+
+def test_sgd_matches_torch_float64(orc):
+    """The SGD fallback: clip_grad_norm_ + torch.optim.SGD(momentum=0,
+    weight_decay=wd) in float64 (coupled decay equals decoupled decay for
+    plain SGD in exact arithmetic)."""
+    rng = np.random.default_rng(31)
+    n1, n2 = 2000, 500
+    lr, wd = float(F32(5e-3)), float(F32(0.1))
+    master = (rng.standard_normal(n1 + n2) * 0.02).astype(np.float32)
+    sh = orc.OracleShard(master, orc.OracleHparams(clip_norm=1.0, init_scale=1.0, scale_window=10 ** 6, optimizer=1),
+                         segments=[(0, n1, wd), (n1, n2, 0.0)])
+    p1 = torch.nn.Parameter(torch.from_numpy(master[:n1].astype(np.float64)))
+    p2 = torch.nn.Parameter(torch.from_numpy(master[n1:].astype(np.float64)))
+    opt = torch.optim.SGD([{"params": [p1], "weight_decay": wd}, {"params": [p2], "weight_decay": 0.0}], lr=lr,
+                          momentum=0.0, foreach=False)
+    for step in range(20):
+        g = f16(rng.standard_normal(n1 + n2) * (0.05 if step % 2 else 1e-3))
+        info = sh.step([g], lr)
+        gd = torch.from_numpy(dec_f16(g))
+        p1.grad, p2.grad = gd[:n1].clone(), gd[n1:].clone()
+        torch.nn.utils.clip_grad_norm_([p1, p2], 1.0, foreach=False)
+        opt.step()
+    ref = torch.cat([p1.detach(), p2.detach()]).numpy()
+    np.testing.assert_allclose(sh.master, ref, rtol=1e-5, atol=1e-7)
+
+
+def test_sgd_closed_form_and_untouched_moments(orc):
+    """wd = 0, clipping off, scale 1: one SGD step is p - lr*g to within the
+    two roundings; m and v stay zero."""
+    n, lr = 5000, 1e-2
+    rng = np.random.default_rng(32)
+    master = (rng.standard_normal(n) * 0.02).astype(np.float32)
+    sh = orc.OracleShard(master, orc.OracleHparams(clip_norm=0.0, init_scale=1.0, optimizer=1), default_wd=0.0)
+    g = f16(rng.standard_normal(n))
+    sh.step([g], lr)
+    expect = master.astype(np.float64) - F32(lr) * dec_f16(g)
+    np.testing.assert_allclose(sh.master, expect, rtol=2.0 ** -22, atol=lr * 2.0 ** -22)
+    assert not sh.m.any() and not sh.v.any()
+    np.testing.assert_array_equal(sh.w, f16(sh.master))
