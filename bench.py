@@ -31,6 +31,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "Adam shard-step Gparams/s and achieved HBM GB/s (% of B200 peak), 1 GPU"
+# the same measurement with the plain-SGD update (a side line, not the headline)
+METRIC_SGD = "SGD shard-step Gparams/s and achieved HBM GB/s (% of B200 peak), 1 GPU"
 UNIT = "Gparams/s"
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SRCS = [os.path.join(ROOT, "mixed_precision_zero_b200", "csrc", f) for f in ("neox_shard.cu", "neox_common.cuh")]
@@ -54,6 +56,8 @@ def parse_args(argv=None):
                    help="flat: neox_shard_step; multi: neox_multi_step with one tensor per segment")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--optimizer", choices=["adamw", "sgd"], default="adamw",
+                   help="update rule of pass 2 (sgd: plain SGD, m and v untouched)")
     a = p.parse_args(argv)
     if a.warmup < 3:
         p.error("--warmup must be >= 3")
@@ -62,10 +66,14 @@ def parse_args(argv=None):
 
 # ------------------------------------------------------------------ workload bytes
 
-def alg_bytes_per_param(K: int, acc: bool):
-    """Algorithmic HBM bytes per parameter of an applied step: (pass 1, pass 2)."""
+def alg_bytes_per_param(K: int, acc: bool, sgd: bool = False):
+    """Algorithmic HBM bytes per parameter of an applied step: (pass 1, pass 2).
+    Pass 2 reads the gradient (K 16-bit buffers, or the FP32 sum) and the FP32
+    state, and writes the state and the 16-bit weight: master/m/v for AdamW,
+    master alone for SGD."""
     p1 = 2 * K + (4 if acc else 0)
-    p2 = (4 if acc else 2 * K) + 12 + 12 + 2
+    state = 4 if sgd else 12
+    p2 = (4 if acc else 2 * K) + state + state + 2
     return p1, p2
 
 
@@ -87,10 +95,10 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
+def recorded_traffic(workload: str, kernel: str = "adam_kernel"):
     """DRAM bytes per launch of the update kernel from the committed ncu summary,
     if it was taken on the current kernel source; else None."""
-    path = os.path.join(ROOT, "profiles", f"adam_kernel_{workload}.md")
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
@@ -217,7 +225,7 @@ def sample_segments(wl, lo, n):
     return segs, inits
 
 
-def run_oracle_sample(wl, n_sample, steps, seconds, rank_seed=0):
+def run_oracle_sample(wl, n_sample, steps, seconds, rank_seed=0, optimizer="adamw"):
     """Time the single-threaded oracle on `steps` calls over a contiguous sample
     of the workload (inputs drawn by the numpy twin of the generator, untimed)."""
     import numpy as np
@@ -233,7 +241,7 @@ def run_oracle_sample(wl, n_sample, steps, seconds, rank_seed=0):
         elif init == "one":
             master[a:a + c] = 1
     hp = oracle.OracleHparams(wl.beta1, wl.beta2, wl.eps, wl.clip, wl.predivide, wl.bench_scale or wl.init_scale,
-                              2.0, 1.0, wl.scale_window)
+                              2.0, 1.0, wl.scale_window, optimizer=1 if optimizer == "sgd" else 0)
     sh = oracle.OracleShard(master, hp, wbf16=wl.bf16, gbf16=wl.bf16, segments=segs, default_wd=wl.weight_decay)
     grads = []
     for k in range(wl.K):
@@ -263,15 +271,15 @@ def run_reference(args):
     total = args.steps + args.warmup
     per_step_budget = max(0.2, 150.0 / total)           # whole run within a few minutes
     n_sample = int(min(1 << 24, max(1 << 16, per_step_budget / 60e-9)))
-    out = run_oracle_sample(wl, n_sample, total, 0.0)
+    out = run_oracle_sample(wl, n_sample, total, 0.0, optimizer=args.optimizer)
     times = out["times"][args.warmup:]
     sec = sum(times)
     value = out["n"] * len(times) / sec / 1e9
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "impl": "reference", "metric": METRIC_SGD if args.optimizer == "sgd" else METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": len(times), "warmup": args.warmup, "ms_per_step": 1e3 * sec / len(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": wl.name, "numel": wl.numel, "grad_buffers": wl.K,
+        "config": {"workload": wl.name, "numel": wl.numel, "grad_buffers": wl.K, "optimizer": args.optimizer,
                    "sample": f"{out['n']} contiguous elements from index {out['lo']} per step"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": f"{out['n']} contiguous elements of {wl.name}, {len(times)} timed steps"},
@@ -291,7 +299,7 @@ def _at_offset(n, dtype, offset):
     return base.narrow(0, offset, n)
 
 
-def build_gpu_workload(wl, rank):
+def build_gpu_workload(wl, rank, optimizer="adamw"):
     import torch
 
     import synth
@@ -320,7 +328,8 @@ def build_gpu_workload(wl, rank):
         else:
             synth.gpu_grad_normal16(g, wl.grad_sigma, scale, seed, k, 1, wl.bf16)
         grads.append(g)
-    hp = Hparams(wl.beta1, wl.beta2, wl.eps, wl.clip, wl.predivide, scale, 2.0, 1.0, wl.scale_window)
+    hp = Hparams(wl.beta1, wl.beta2, wl.eps, wl.clip, wl.predivide, scale, 2.0, 1.0, wl.scale_window,
+                 optimizer=optimizer)
     shard = NeoxShard(master, m, v, hp, wdtype=dt, gdtype=dt, segments=wl.seg_table(),
                       weight_decay=wl.weight_decay, max_grads=wl.K)
     torch.cuda.synchronize()
@@ -340,7 +349,8 @@ def run_multi(args):
     shard.close()
     segs = wl.seg_table() or [(0, wl.numel, wl.weight_decay)]
     scale = wl.bench_scale or wl.init_scale
-    hp = Hparams(wl.beta1, wl.beta2, wl.eps, wl.clip, wl.predivide, scale, 2.0, 1.0, wl.scale_window)
+    hp = Hparams(wl.beta1, wl.beta2, wl.eps, wl.clip, wl.predivide, scale, 2.0, 1.0, wl.scale_window,
+                 optimizer=args.optimizer)
     multi = NeoxMultiShard([{"master": master[o:o + c], "exp_avg": m[o:o + c], "exp_avg_sq": v[o:o + c],
                              "params": params[o:o + c], "grads": [g[o:o + c] for g in grads], "weight_decay": w}
                             for o, c, w in segs], hp)
@@ -357,12 +367,13 @@ def run_multi(args):
         torch.cuda.synchronize()
     assert multi.get_state()[2] - t0 == args.steps
     ms = e0.elapsed_time(e1)
-    p1b, p2b = alg_bytes_per_param(wl.K, False)
+    p1b, p2b = alg_bytes_per_param(wl.K, False, args.optimizer == "sgd")
     peak, kind = hbm_peak()
-    line = {"metric": METRIC, "value": wl.numel * args.steps / (ms * 1e-3) / 1e9, "unit": UNIT, "n_gpus": 1,
+    line = {"metric": METRIC_SGD if args.optimizer == "sgd" else METRIC, "value": wl.numel * args.steps / (ms * 1e-3) / 1e9, "unit": UNIT, "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "impl": "b200",
-            "config": {"workload": wl.name, "api": "neox_multi_step", "tensors": len(segs)},
+            "config": {"workload": wl.name, "api": "neox_multi_step", "tensors": len(segs),
+                       "optimizer": args.optimizer},
             "hbm": {"step_gbs": (p1b + p2b) * wl.numel / (ms / args.steps * 1e-3) / 1e9,
                     "step_frac": (p1b + p2b) * wl.numel / (ms / args.steps * 1e-3) / 1e9 / peak, "peak_gbs": peak,
                     "peak_kind": kind},
@@ -386,9 +397,11 @@ def run_b200(args):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
     wl = W.ALL[args.workload]()
-    shard, grads, params, state = build_gpu_workload(wl, rank)
+    sgd = args.optimizer == "sgd"
+    shard, grads, params, state = build_gpu_workload(wl, rank, args.optimizer)
     acc = wl.K >= 5
-    p1b, p2b = alg_bytes_per_param(wl.K, acc)
+    p1b, p2b = alg_bytes_per_param(wl.K, acc, sgd)
+    kernel2 = "sgd_kernel" if sgd else "adam_kernel"
     stream = torch.cuda.current_stream()
 
     # One step.  A single GPU runs the fused step; several ranks run the split
@@ -440,7 +453,7 @@ def run_b200(args):
     peak, peak_kind = hbm_peak()
     achieved = p2b * wl.numel / (p2_ms * 1e-3) / 1e9
     step_gbs = (p1b + p2b) * wl.numel / (ms_local / args.steps * 1e-3) / 1e9
-    traffic = recorded_traffic(args.workload)
+    traffic = recorded_traffic(args.workload, kernel2)
 
     # the same step through the asynchronous entry point, captured once in a
     # CUDA graph and replayed (no host synchronisation between steps)
@@ -497,7 +510,7 @@ def run_b200(args):
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        out = run_oracle_sample(wl, 1 << 25, 50, args.cpu_seconds)
+        out = run_oracle_sample(wl, 1 << 25, 50, args.cpu_seconds, optimizer=args.optimizer)
         sec = sum(out["times"])
         cpu = {"value": out["n"] * len(out["times"]) / sec / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": f"{len(out['times'])} steps over {out['n']} contiguous elements of {wl.name} "
@@ -505,19 +518,20 @@ def run_b200(args):
 
     clk = clocks.summary()
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "metric": METRIC_SGD if sgd else METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic",
         "config": {"workload": wl.name, "numel_per_rank": wl.numel, "segments": len(wl.segments or [1]),
                    "grad_buffers": wl.K, "weights": "bf16" if wl.bf16 else "fp16",
                    "element_offset": wl.elem_offset, "loss_scale": wl.bench_scale or wl.init_scale,
-                   "state": "fp32 master/m/v",
-                   "l2": f"inputs {(14 + 2 * wl.K) * wl.numel / 1e9:.1f} GB per rank >> 126 MB L2; no flush",
+                   "state": "fp32 master/m/v", "optimizer": args.optimizer,
+                   "l2": f"inputs {((6 if sgd else 14) + 2 * wl.K) * wl.numel / 1e9:.1f} GB per rank >> 126 MB L2; "
+                         "no flush",
                    "parallelism": (f"dp{ws}: one shard per GPU, 16-byte NCCL all-reduce of the pass-1 statistics "
                                    "per step" if split else "one shard on one GPU")},
         "hbm": {"step_gbs": step_gbs, "step_frac": step_gbs / peak, "bytes_per_param": p1b + p2b,
                 "peak_gbs": peak, "peak_kind": peak_kind},
-        "roofline": {"bound": "hbm", "kernel": "adam_kernel (pass 2)", "achieved": achieved, "peak": peak,
+        "roofline": {"bound": "hbm", "kernel": f"{kernel2} (pass 2)", "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
                      "traffic": traffic, "alg_bytes_per_launch": p2b * wl.numel,
                      "avg_launch_ms": p2_ms, "grad_pass_avg_ms": p1_ms},

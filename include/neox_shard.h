@@ -25,12 +25,19 @@
  *      post = K/predivide, the sum taken in buffer order in FP32;
  *   2. overflow = any g_i not finite (or the norm not finite);
  *   3. norm = sqrt(sum_i g_i^2)  (pre-clip, unscaled);
- *   4. loss scaler: overflow -> S = max(S/factor, min_scale), counter = 0, skip;
- *      applied -> counter+1, at scale_window S = S*factor (if finite), counter = 0;
+ *   4. loss scaler: overflow -> counter = 0, skip, and the hysteresis count
+ *      H drops by one (not below 0); when it is 0, S = max(S/factor,
+ *      min_scale); applied -> counter+1, at scale_window S = S*factor (if
+ *      finite), counter = 0, H = max(hysteresis, 1).  With hysteresis 0 or 1
+ *      every overflow lowers the scale;
  *   5. unless skipped: t = t+1; c = clip/(norm+1e-6) if that is < 1 (else 1);
  *      for every element: gh = g*c; m = b1*m + (1-b1)*gh; v = b2*v + (1-b2)*gh*gh;
  *      p = p*(1 - lr*wd_seg) - (lr/bc1) * m / (sqrt(v)/sqrt(bc2) + eps),
  *      bc1 = 1-b1^t, bc2 = 1-b2^t; w = RNE16(p).
+ *      With optimizer = NEOX_SGD the update is instead plain SGD with the
+ *      same decoupled decay, p = p*(1 - lr*wd_seg) - lr*gh, and m, v are
+ *      neither read nor written (same page, "方法适配": SGD was tried in
+ *      place of Adam).
  *
  * Threading: a handle is used by one host thread at a time.  Different
  * handles are independent.  All functions are host functions.
@@ -63,6 +70,9 @@ typedef struct {
     float weight_decay;
 } neox_segment;
 
+/* The update rule of pass 2. */
+typedef enum { NEOX_ADAMW = 0, NEOX_SGD = 1 } neox_optimizer;
+
 typedef struct {
     float beta1, beta2;   /* in [0, 1)                                      */
     float eps;            /* >= 0                                           */
@@ -73,6 +83,10 @@ typedef struct {
     float scale_factor;   /* >= 1: backoff divisor and growth multiplier    */
     float min_scale;      /* >= 0: floor of the scale after a backoff       */
     int32_t scale_window; /* >= 1: applied steps between growths            */
+    int32_t hysteresis;   /* >= 0: overflows since the last growth (or
+                             create / set_state) before the scale is
+                             lowered; 0 or 1 = at every overflow           */
+    int32_t optimizer;    /* neox_optimizer; 0 = NEOX_ADAMW                 */
 } neox_hparams;
 
 /* The shard.  numel may be 0 (a rank that owns nothing still takes part in
@@ -194,14 +208,42 @@ neox_status neox_shard_grad_stats(neox_shard* h, const void* const* grads, int32
 neox_status neox_shard_apply(neox_shard* h, const void* const* grads, int32_t num_grads, void* params, float lr,
                              const double* stats_device, void* cuda_stream, neox_step_result* out);
 
-/* Replace the hyperparameters (e.g. the clip 1.0 -> 0.3 change); the current
- * loss scale and counters are kept (init_scale is ignored here). */
+/* Extra destinations of the updated 16-bit working weights, written by pass 2
+ * with the same bytes as `params` (and never on a skipped step).  Under ZeRO
+ * the updated weight shards are all-gathered to every rank ("GPT-NeoX: how it
+ * opened the door to democratised 100B-scale training" (ainews.cool),
+ * "技术深度解析": reduce-scatter / all-gather); given, for each peer, a
+ * peer-mapped pointer to this rank's slice of that peer's full-weight buffer
+ * (CUDA IPC or peer access over NVLink), the cast itself performs that
+ * all-gather with direct stores, with no separate collective.  Any
+ * device-accessible memory works (local buffers too).
+ *   dsts: host array of n device pointers (2-byte aligned), n in [0, 8];
+ *         n = 0 removes the copies.  Each destination receives numel elements.
+ * The pointers must stay valid for every later step; the vector layout takes
+ * them into account (a destination with another residue mod 16 bytes makes
+ * the kernels use narrower vectors). */
+neox_status neox_shard_set_weight_copies(neox_shard* h, void* const* dsts, int32_t n);
+
+/* Replace the hyperparameters (e.g. the clip 1.0 -> 0.3 change, or a switch
+ * to NEOX_SGD); the current loss scale and counters are kept (init_scale is
+ * ignored here), and so is the hysteresis count, which takes a new
+ * `hysteresis` at the next growth or set_state.  Switching the optimizer
+ * leaves m and v as they are. */
 neox_status neox_shard_set_hparams(neox_shard* h, const neox_hparams* hp);
 
 /* Scaler / step-count state, for checkpoint and resume.  Any pointer may be
- * NULL.  set_state validates scale > 0 finite, good >= 0, t >= 0. */
+ * NULL.  set_state validates scale > 0 finite, good >= 0, t >= 0, and resets
+ * the hysteresis count to max(hysteresis, 1): it is the loss-scaler reset of
+ * the OPT summary, "方法适配". */
 neox_status neox_shard_get_state(const neox_shard* h, float* scale, int32_t* good, int64_t* t);
 neox_status neox_shard_set_state(neox_shard* h, float scale, int32_t good, int64_t t);
+
+/* The hysteresis count H of step 4 (overflows still tolerated before the next
+ * back-off), for an exact checkpoint: set it after set_state on resume.
+ * set_hysteresis validates count >= 0.  Waits for asynchronous steps as
+ * get_state / set_state do. */
+neox_status neox_shard_get_hysteresis(const neox_shard* h, int32_t* count);
+neox_status neox_shard_set_hysteresis(neox_shard* h, int32_t count);
 
 /* Free what create allocated (never the caller's arrays).  NULL is a no-op. */
 void neox_shard_destroy(neox_shard* h);
@@ -291,6 +333,8 @@ neox_status neox_multi_rebind_grads(neox_multi* h, const void* const* grads);
 neox_status neox_multi_set_hparams(neox_multi* h, const neox_hparams* hp);
 neox_status neox_multi_get_state(const neox_multi* h, float* scale, int32_t* good, int64_t* t);
 neox_status neox_multi_set_state(neox_multi* h, float scale, int32_t good, int64_t t);
+neox_status neox_multi_get_hysteresis(const neox_multi* h, int32_t* count);
+neox_status neox_multi_set_hysteresis(neox_multi* h, int32_t count);
 void neox_multi_destroy(neox_multi* h);
 const char* neox_multi_last_error(const neox_multi* h);
 
@@ -313,6 +357,8 @@ const char* neox_multi_last_error(const neox_multi* h);
  * NEOX_ERR_INVALID_ARGUMENT and a message); K in [1, 64].  There is no FP32
  * gradient-sum buffer (it would need numel*4 bytes), so K >= 5 re-reads the K
  * buffers in pass 2; desc->max_grads is ignored.  numel itself is not limited.
+ * The scaler state below has no hysteresis count, so hp->hysteresis must be
+ * 0 or 1 (a larger value is rejected); hp->optimizer is honoured.
  *
  * Arguments are those of neox_shard_create + neox_shard_step; desc->numel,
  * dtypes, segment table and the caller-owned master / exp_avg / exp_avg_sq

@@ -24,7 +24,9 @@ from ._abi import (NEOX_BF16, NEOX_ERR_CUDA, NEOX_ERR_INVALID_ARGUMENT, NEOX_ERR
                    neox_shard_step, neox_shard_step_async, neox_status_string, neox_step_result,
                    neox_tensor, neox_tensor_set, neox_multi_create, neox_multi_step, neox_multi_step_async,
                    neox_multi_rebind_grads, neox_multi_get_state, neox_multi_set_state,
-                   neox_multi_set_hparams, neox_multi_destroy, neox_shard_grad_stats, neox_shard_apply)
+                   neox_multi_set_hparams, neox_multi_destroy, neox_shard_grad_stats, neox_shard_apply,
+                   neox_shard_set_weight_copies, neox_shard_get_hysteresis, neox_shard_set_hysteresis,
+                   neox_multi_get_hysteresis, neox_multi_set_hysteresis, NEOX_ADAMW, NEOX_SGD)
 
 __all__ = ["NeoxShard", "NeoxMultiShard", "Hparams", "NeoxError", "neox_shard_create", "neox_shard_step",
            "neox_shard_destroy", "neox_shard_set_hparams", "neox_shard_get_state",
@@ -42,10 +44,16 @@ class Hparams:
     scale_factor: float = 2.0
     min_scale: float = 1.0
     scale_window: int = 1000
+    hysteresis: int = 1          # overflows before a back-off (0 or 1: at every overflow)
+    optimizer: str = "adamw"     # "adamw" or "sgd"
 
     def c(self) -> neox_hparams:
+        opts = {"adamw": NEOX_ADAMW, "sgd": NEOX_SGD}
+        if self.optimizer not in opts:
+            raise ValueError(f"optimizer must be 'adamw' or 'sgd', got {self.optimizer!r}")
         return neox_hparams(self.beta1, self.beta2, self.eps, self.clip_norm, self.predivide,
-                            self.init_scale, self.scale_factor, self.min_scale, self.scale_window)
+                            self.init_scale, self.scale_factor, self.min_scale, self.scale_window,
+                            self.hysteresis, opts[self.optimizer])
 
 
 def _dtype_code(t) -> int:
@@ -138,6 +146,16 @@ class NeoxShard:
         sp = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
         return neox_shard_apply(self.handle, [g.data_ptr() for g in grads], params.data_ptr(), lr, stats.data_ptr(), sp)
 
+    def set_weight_copies(self, dsts) -> None:
+        """Extra 16-bit tensors (same length and type as params) that pass 2
+        writes with the updated weights, e.g. peer-mapped slices of every
+        rank's full-weight buffer.  An empty list removes them."""
+        for d in dsts:
+            if d.numel() != self.numel or _dtype_code(d) != self.wdtype or not d.is_contiguous():
+                raise ValueError("each copy must be a contiguous 16-bit tensor like params")
+        self._copies = list(dsts)  # keep them alive
+        neox_shard_set_weight_copies(self.handle, [d.data_ptr() for d in dsts])
+
     def set_hparams(self, hp: Hparams) -> None:
         neox_shard_set_hparams(self.handle, hp.c())
 
@@ -146,6 +164,12 @@ class NeoxShard:
 
     def set_state(self, scale: float, good: int, t: int) -> None:
         neox_shard_set_state(self.handle, scale, good, t)
+
+    def get_hysteresis(self) -> int:
+        return neox_shard_get_hysteresis(self.handle)
+
+    def set_hysteresis(self, count: int) -> None:
+        neox_shard_set_hysteresis(self.handle, count)
 
     def set_profiling(self, enable: bool) -> None:
         neox_shard_set_profiling(self.handle, enable)
@@ -233,6 +257,12 @@ class NeoxMultiShard:
 
     def set_state(self, scale: float, good: int, t: int) -> None:
         neox_multi_set_state(self.handle, scale, good, t)
+
+    def get_hysteresis(self) -> int:
+        return neox_multi_get_hysteresis(self.handle)
+
+    def set_hysteresis(self, count: int) -> None:
+        neox_multi_set_hysteresis(self.handle, count)
 
     def set_hparams(self, hp: Hparams) -> None:
         neox_multi_set_hparams(self.handle, hp.c())

@@ -20,6 +20,9 @@ NEOX_ERR_UNSUPPORTED = 4
 NEOX_FP16 = 0
 NEOX_BF16 = 1
 
+NEOX_ADAMW = 0
+NEOX_SGD = 1
+
 
 class neox_segment(ctypes.Structure):
     _fields_ = [("offset", ctypes.c_uint64), ("numel", ctypes.c_uint64), ("weight_decay", ctypes.c_float)]
@@ -29,7 +32,8 @@ class neox_hparams(ctypes.Structure):
     _fields_ = [("beta1", ctypes.c_float), ("beta2", ctypes.c_float), ("eps", ctypes.c_float),
                 ("clip_norm", ctypes.c_float), ("predivide", ctypes.c_float),
                 ("init_scale", ctypes.c_float), ("scale_factor", ctypes.c_float),
-                ("min_scale", ctypes.c_float), ("scale_window", ctypes.c_int32)]
+                ("min_scale", ctypes.c_float), ("scale_window", ctypes.c_int32),
+                ("hysteresis", ctypes.c_int32), ("optimizer", ctypes.c_int32)]
 
 
 class neox_shard_desc(ctypes.Structure):
@@ -99,6 +103,8 @@ def lib() -> ctypes.CDLL:
                                        ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
                                        ctypes.POINTER(neox_step_result)]
         L.neox_shard_apply.restype = S
+        L.neox_shard_set_weight_copies.argtypes = [_H, ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]
+        L.neox_shard_set_weight_copies.restype = S
         L.neox_shard_set_hparams.argtypes = [_H, ctypes.POINTER(neox_hparams)]
         L.neox_shard_set_hparams.restype = S
         L.neox_shard_get_state.argtypes = [_H, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int32),
@@ -106,6 +112,10 @@ def lib() -> ctypes.CDLL:
         L.neox_shard_get_state.restype = S
         L.neox_shard_set_state.argtypes = [_H, ctypes.c_float, ctypes.c_int32, ctypes.c_int64]
         L.neox_shard_set_state.restype = S
+        L.neox_shard_get_hysteresis.argtypes = [_H, ctypes.POINTER(ctypes.c_int32)]
+        L.neox_shard_get_hysteresis.restype = S
+        L.neox_shard_set_hysteresis.argtypes = [_H, ctypes.c_int32]
+        L.neox_shard_set_hysteresis.restype = S
         L.neox_shard_destroy.argtypes = [_H]
         L.neox_shard_destroy.restype = None
         L.neox_status_string.argtypes = [S]
@@ -143,6 +153,10 @@ def lib() -> ctypes.CDLL:
         L.neox_multi_get_state.restype = S
         L.neox_multi_set_state.argtypes = [_H, ctypes.c_float, ctypes.c_int32, ctypes.c_int64]
         L.neox_multi_set_state.restype = S
+        L.neox_multi_get_hysteresis.argtypes = [_H, ctypes.POINTER(ctypes.c_int32)]
+        L.neox_multi_get_hysteresis.restype = S
+        L.neox_multi_set_hysteresis.argtypes = [_H, ctypes.c_int32]
+        L.neox_multi_set_hysteresis.restype = S
         L.neox_multi_destroy.argtypes = [_H]
         L.neox_multi_destroy.restype = None
         L.neox_multi_last_error.argtypes = [_H]
@@ -218,6 +232,20 @@ def neox_shard_get_state(h: int):
 
 def neox_shard_set_state(h: int, scale: float, good: int, t: int) -> None:
     st = lib().neox_shard_set_state(h, scale, good, t)
+    if st != NEOX_OK:
+        raise NeoxError(st, lib().neox_last_error(h).decode())
+
+
+def neox_shard_get_hysteresis(h: int) -> int:
+    c = ctypes.c_int32()
+    st = lib().neox_shard_get_hysteresis(h, ctypes.byref(c))
+    if st != NEOX_OK:
+        raise NeoxError(st, lib().neox_last_error(h).decode())
+    return c.value
+
+
+def neox_shard_set_hysteresis(h: int, count: int) -> None:
+    st = lib().neox_shard_set_hysteresis(h, count)
     if st != NEOX_OK:
         raise NeoxError(st, lib().neox_last_error(h).decode())
 
@@ -317,6 +345,20 @@ def neox_multi_set_state(h: int, scale: float, good: int, t: int) -> None:
         raise NeoxError(st, _merr(h))
 
 
+def neox_multi_get_hysteresis(h: int) -> int:
+    c = ctypes.c_int32()
+    st = lib().neox_multi_get_hysteresis(h, ctypes.byref(c))
+    if st != NEOX_OK:
+        raise NeoxError(st, _merr(h))
+    return c.value
+
+
+def neox_multi_set_hysteresis(h: int, count: int) -> None:
+    st = lib().neox_multi_set_hysteresis(h, count)
+    if st != NEOX_OK:
+        raise NeoxError(st, _merr(h))
+
+
 def neox_multi_set_hparams(h: int, hp: neox_hparams) -> None:
     st = lib().neox_multi_set_hparams(h, ctypes.byref(hp))
     if st != NEOX_OK:
@@ -325,3 +367,10 @@ def neox_multi_set_hparams(h: int, hp: neox_hparams) -> None:
 
 def neox_multi_destroy(h: int) -> None:
     lib().neox_multi_destroy(h)
+
+
+def neox_shard_set_weight_copies(h: int, dst_ptrs) -> None:
+    arr = (ctypes.c_void_p * max(1, len(dst_ptrs)))(*dst_ptrs)
+    st = lib().neox_shard_set_weight_copies(h, arr, len(dst_ptrs))
+    if st != NEOX_OK:
+        raise NeoxError(st, lib().neox_last_error(h).decode())

@@ -49,7 +49,8 @@ struct __align__(64) DevScalars {
     float step_size;       // device-computed fl32(lr / bc1) of the last step (asynchronous steps)
     float bc2_sqrt;        // device-computed fl32(sqrt(bc2)) of the last step (asynchronous steps)
     float lr;              // learning rate of the last step (asynchronous steps)
-    int32_t pad_[2];
+    int32_t hyst;          // overflows still tolerated before the next back-off
+    int32_t pad_;
 };
 static_assert(sizeof(DevScalars) == 64, "DevScalars is one 64-byte block");
 
@@ -65,6 +66,7 @@ struct ScalerArgs {
     float clip;           // <= 0: off
     float factor, min_scale;
     int32_t window;
+    int32_t hyst_full;    // max(hysteresis, 1): the count after a growth
     // asynchronous steps: the bias corrections are formed on the device from
     // the device step count, and the result is written to `result`
     int32_t device_bc;
@@ -74,6 +76,15 @@ struct ScalerArgs {
     // split step: pass 1 writes {sum of squares, non-finite flag} here and
     // takes no decision (the ranks' statistics are all-reduced first)
     double* stats_out;
+};
+
+// Extra destinations of the 16-bit working weights (e.g. this rank's slice
+// of the full weight buffer on every peer), written with the same bytes as
+// the shard's own copy.
+constexpr int kMaxWeightCopies = 8;
+struct WeightCopies {
+    uint16_t* p[kMaxWeightCopies];
+    int n;
 };
 
 struct AdamArgs {
@@ -338,8 +349,13 @@ __device__ __forceinline__ void decide_step(DevScalars* __restrict__ sc, const S
     sc->sumsq = s;
     sc->overflow = overflow;
     if (overflow) {
-        const float d = S / sa.factor;
-        S = d > sa.min_scale ? d : sa.min_scale;
+        int h = sc->hyst;
+        if (h > 0) h -= 1;
+        sc->hyst = h;
+        if (h == 0) {
+            const float d = S / sa.factor;
+            S = d > sa.min_scale ? d : sa.min_scale;
+        }
         good = 0;
         sc->coef = 0.0f;
         sc->norm = __int_as_float(0x7f800000);
@@ -349,6 +365,7 @@ __device__ __forceinline__ void decide_step(DevScalars* __restrict__ sc, const S
             const float u = S * sa.factor;
             if (!not_finite(u)) S = u;
             good = 0;
+            sc->hyst = sa.hyst_full;
         }
         t += 1;
         float c = 1.0f;
@@ -445,6 +462,17 @@ __device__ __forceinline__ void adam_vec(const float (&g)[VEC], const float (&ke
     }
 }
 
+// Plain SGD (no momentum) with the decoupled decay: p*keep - lr*(g*c).
+template <int VEC>
+__device__ __forceinline__ void sgd_vec(const float (&g)[VEC], const float (&keep)[VEC], float c, float lr,
+                                        float (&p)[VEC]) {
+#pragma unroll
+    for (int e = 0; e < VEC; e++) {
+        const float gh = __fmul_rn(g[e], c);
+        p[e] = __fsub_rn(__fmul_rn(p[e], keep[e]), __fmul_rn(lr, gh));
+    }
+}
+
 // The decision of a split step from all-reduced statistics {sum of squares,
 // number of ranks that saw a non-finite value}.  One thread.
 __global__ void decide_kernel(DevScalars* __restrict__ sc, ScalerArgs sa, const double* __restrict__ stats) {
@@ -479,7 +507,47 @@ const char* check_hparams(const neox_hparams* hp) {
     if (!(hp->scale_factor >= 1.0f) || !finite(hp->scale_factor)) return "scale_factor must be finite and >= 1";
     if (!(hp->min_scale >= 0.0f) || !finite(hp->min_scale)) return "min_scale must be finite and >= 0";
     if (hp->scale_window < 1) return "scale_window must be >= 1";
+    if (hp->hysteresis < 0) return "hysteresis must be >= 0";
+    if (hp->optimizer != NEOX_ADAMW && hp->optimizer != NEOX_SGD) return "optimizer must be NEOX_ADAMW or NEOX_SGD";
     return nullptr;
+}
+
+int hyst_full(const neox_hparams& hp) { return hp.hysteresis > 1 ? hp.hysteresis : 1; }
+
+// The launch arguments of one step over K buffers.  device_bc = false: the
+// bias corrections for step t+1 are formed here in double (the step count if
+// this step is applied); true: the last pass-1 block forms them on the device.
+void make_step_args(const neox_hparams& hp, int K, float lr, long long t, bool device_bc, ScalerArgs& sa,
+                    AdamArgs& a) {
+    sa = ScalerArgs{};
+    sa.post = (double)K / (double)hp.predivide;
+    sa.inv_pre = (float)(1.0 / (double)hp.predivide);
+    sa.clip = hp.clip_norm;
+    sa.factor = hp.scale_factor;
+    sa.min_scale = hp.min_scale;
+    sa.window = hp.scale_window;
+    sa.hyst_full = hyst_full(hp);
+    sa.device_bc = device_bc ? 1 : 0;
+    sa.lr = lr;
+    sa.beta1 = hp.beta1;
+    sa.beta2 = hp.beta2;
+    a = AdamArgs{};
+    a.lr = lr;
+    a.b1 = hp.beta1;
+    a.b2 = hp.beta2;
+    a.omb1 = 1.0f - hp.beta1;
+    a.omb2 = 1.0f - hp.beta2;
+    a.eps = hp.eps;
+    if (!device_bc) {
+        const double t1 = (double)(t + 1);
+        const double bc1 = 1.0 - std::pow((double)hp.beta1, t1);
+        const double bc2 = 1.0 - std::pow((double)hp.beta2, t1);
+        a.step_size = (float)((double)lr / bc1);
+        a.bcs = (float)std::sqrt(bc2);
+    }
+    a.device_bc = device_bc ? 1 : 0;
+    a.inv_pre = sa.inv_pre;
+    a.post = sa.post;
 }
 
 int elem_size(neox_dtype) { return 2; }

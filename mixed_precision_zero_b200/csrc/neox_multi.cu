@@ -138,7 +138,7 @@ mt_stats_kernel(const MtTensor* __restrict__ tens, int ntensors, const uint16_t*
 }
 
 // ---------------------------------------------------------------- pass 2
-template <class G, class W, int VEC, int KFIX>
+template <bool SGD, class G, class W, int VEC, int KFIX>
 __device__ __forceinline__ void mt_p2_tensor(const GradTab& gp, int K_rt, const MtTensor& T, float keep1, float c,
                                              float inv_us, const AdamArgs& a) {
     const int K = KFIX ? KFIX : K_rt;
@@ -156,31 +156,37 @@ __device__ __forceinline__ void mt_p2_tensor(const GradTab& gp, int K_rt, const 
         float g[VEC], p[VEC], mm[VEC], vv[VEC];
         ingest<G, VEC>(gp, K, i, a.inv_pre, inv_us, g);
         ld32<VEC>(master + i, p);
-        ld32<VEC>(m + i, mm);
-        ld32<VEC>(v + i, vv);
-        adam_vec<VEC>(g, keep, c, a, p, mm, vv);
-        st32<VEC>(master + i, p);
-        st32<VEC>(m + i, mm);
-        st32<VEC>(v + i, vv);
+        if constexpr (SGD) {
+            sgd_vec<VEC>(g, keep, c, a.lr, p);
+            st32<VEC>(master + i, p);
+        } else {
+            ld32<VEC>(m + i, mm);
+            ld32<VEC>(v + i, vv);
+            adam_vec<VEC>(g, keep, c, a, p, mm, vv);
+            st32<VEC>(master + i, p);
+            st32<VEC>(m + i, mm);
+            st32<VEC>(v + i, vv);
+        }
         st16<W, VEC>(w + i, p);
     }
 }
 
-template <class G, class W, int KFIX>
+template <bool SGD, class G, class W, int KFIX>
 __device__ __forceinline__ void mt_p2_dispatch(const MtTensor& T, const GradTab& gp, int K, float keep1, float c,
                                                float inv_us, const AdamArgs& a) {
     switch (T.vec) {
-        case 8: mt_p2_tensor<G, W, 8, KFIX>(gp, K, T, keep1, c, inv_us, a); break;
-        case 4: mt_p2_tensor<G, W, 4, KFIX>(gp, K, T, keep1, c, inv_us, a); break;
-        case 2: mt_p2_tensor<G, W, 2, KFIX>(gp, K, T, keep1, c, inv_us, a); break;
-        default: mt_p2_tensor<G, W, 1, KFIX>(gp, K, T, keep1, c, inv_us, a); break;
+        case 8: mt_p2_tensor<SGD, G, W, 8, KFIX>(gp, K, T, keep1, c, inv_us, a); break;
+        case 4: mt_p2_tensor<SGD, G, W, 4, KFIX>(gp, K, T, keep1, c, inv_us, a); break;
+        case 2: mt_p2_tensor<SGD, G, W, 2, KFIX>(gp, K, T, keep1, c, inv_us, a); break;
+        default: mt_p2_tensor<SGD, G, W, 1, KFIX>(gp, K, T, keep1, c, inv_us, a); break;
     }
 }
 
-template <class G, class W>
-__global__ void __launch_bounds__(kMtThreads3)
-mt_adam_kernel(const MtTensor* __restrict__ tens, int ntensors, const uint16_t* const* __restrict__ gtab, int K,
-               AdamArgs a_arg, const DevScalars* __restrict__ sc) {
+// The whole of pass 2 over every tensor (SGD: plain SGD, else AdamW).
+template <bool SGD, class G, class W>
+__device__ __forceinline__ void mt_update(const MtTensor* __restrict__ tens, int ntensors,
+                                          const uint16_t* const* __restrict__ gtab, int K, const AdamArgs& a_arg,
+                                          const DevScalars* __restrict__ sc) {
     asm volatile("griddepcontrol.wait;" ::: "memory");  // pass 1's results
     if (sc->overflow) return;
     const float c = sc->coef;
@@ -203,23 +209,52 @@ mt_adam_kernel(const MtTensor* __restrict__ tens, int ntensors, const uint16_t* 
         if (T.numel == 0) continue;
         const GradTab gp{gtab, T.gbase};
         const float keep1 = __fsub_rn(1.0f, __fmul_rn(a.lr, T.wd));  // fl32(1 - fl32(lr * wd))
-        if (K == 1) mt_p2_dispatch<G, W, 1>(T, gp, K, keep1, c, inv_us, a);
-        else mt_p2_dispatch<G, W, 0>(T, gp, K, keep1, c, inv_us, a);
+        if (K == 1) mt_p2_dispatch<SGD, G, W, 1>(T, gp, K, keep1, c, inv_us, a);
+        else mt_p2_dispatch<SGD, G, W, 0>(T, gp, K, keep1, c, inv_us, a);
         if ((unsigned)ti % gridDim.x == blockIdx.x) {  // this tensor's head and tail
             const unsigned long long extra = T.head + (T.numel - T.tail0);
             for (unsigned long long j = threadIdx.x; j < extra; j += kMtThreads3) {
                 const unsigned long long i = j < T.head ? j : T.tail0 + (j - T.head);
-                float g[1], p[1] = {T.master[i]}, mm[1] = {T.m[i]}, vv[1] = {T.v[i]}, keep[1] = {keep1};
+                float g[1], p[1] = {T.master[i]}, keep[1] = {keep1};
                 ingest<G, 1>(gp, K, i, a.inv_pre, inv_us, g);
-                adam_vec<1>(g, keep, c, a, p, mm, vv);
+                if constexpr (SGD) {
+                    sgd_vec<1>(g, keep, c, a.lr, p);
+                } else {
+                    float mm[1] = {T.m[i]}, vv[1] = {T.v[i]};
+                    adam_vec<1>(g, keep, c, a, p, mm, vv);
+                    T.m[i] = mm[0];
+                    T.v[i] = vv[0];
+                }
                 T.master[i] = p[0];
-                T.m[i] = mm[0];
-                T.v[i] = vv[0];
                 T.w[i] = W::enc(p[0]);
             }
         }
     }
     }
+}
+
+template <class G, class W>
+__global__ void __launch_bounds__(kMtThreads3)
+mt_adam_kernel(const MtTensor* __restrict__ tens, int ntensors, const uint16_t* const* __restrict__ gtab, int K,
+               AdamArgs a, const DevScalars* __restrict__ sc) {
+    mt_update<false, G, W>(tens, ntensors, gtab, K, a, sc);
+}
+
+template <class G, class W>
+__global__ void __launch_bounds__(kMtThreads3)
+mt_sgd_kernel(const MtTensor* __restrict__ tens, int ntensors, const uint16_t* const* __restrict__ gtab, int K,
+              AdamArgs a, const DevScalars* __restrict__ sc) {
+    mt_update<true, G, W>(tens, ntensors, gtab, K, a, sc);
+}
+
+using MtUpdateKernel = void (*)(const MtTensor*, int, const uint16_t* const*, int, AdamArgs, const DevScalars*);
+
+MtUpdateKernel mt_update_kernel(bool sgd, neox_dtype gdt, neox_dtype wdt) {
+    if (sgd)
+        return gdt == NEOX_FP16 ? (wdt == NEOX_FP16 ? mt_sgd_kernel<F16, F16> : mt_sgd_kernel<F16, BF16>)
+                                : (wdt == NEOX_FP16 ? mt_sgd_kernel<BF16, F16> : mt_sgd_kernel<BF16, BF16>);
+    return gdt == NEOX_FP16 ? (wdt == NEOX_FP16 ? mt_adam_kernel<F16, F16> : mt_adam_kernel<F16, BF16>)
+                            : (wdt == NEOX_FP16 ? mt_adam_kernel<BF16, F16> : mt_adam_kernel<BF16, BF16>);
 }
 
 }  // namespace
@@ -332,36 +367,11 @@ neox_status mt_enqueue(neox_multi* h, float lr, const float* lr_dev, cudaStream_
     if (!lr_dev && (!finite(lr) || lr < 0.0f)) return mfail(h, NEOX_ERR_INVALID_ARGUMENT, "lr must be finite and >= 0");
     if (result && ((uintptr_t)result & 7u)) return mfail(h, NEOX_ERR_INVALID_ARGUMENT, "result must be 8-byte aligned");
     if (lr_dev && ((uintptr_t)lr_dev & 3u)) return mfail(h, NEOX_ERR_INVALID_ARGUMENT, "lr_device must be 4-byte aligned");
-    ScalerArgs sa{};
-    sa.post = (double)h->K / (double)h->hp.predivide;
-    sa.inv_pre = (float)(1.0 / (double)h->hp.predivide);
-    sa.clip = h->hp.clip_norm;
-    sa.factor = h->hp.scale_factor;
-    sa.min_scale = h->hp.min_scale;
-    sa.window = h->hp.scale_window;
-    sa.device_bc = device_bc ? 1 : 0;
-    sa.lr = lr;
-    sa.beta1 = h->hp.beta1;
-    sa.beta2 = h->hp.beta2;
+    ScalerArgs sa;
+    AdamArgs a;
+    make_step_args(h->hp, h->K, lr, h->t, device_bc, sa, a);
     sa.lr_ptr = lr_dev;
     sa.result = result;
-    AdamArgs a{};
-    a.lr = lr;
-    a.b1 = h->hp.beta1;
-    a.b2 = h->hp.beta2;
-    a.omb1 = 1.0f - h->hp.beta1;
-    a.omb2 = 1.0f - h->hp.beta2;
-    a.eps = h->hp.eps;
-    if (!device_bc) {
-        const double t1 = (double)(h->t + 1);
-        const double bc1 = 1.0 - std::pow((double)h->hp.beta1, t1);
-        const double bc2 = 1.0 - std::pow((double)h->hp.beta2, t1);
-        a.step_size = (float)((double)lr / bc1);
-        a.bcs = (float)std::sqrt(bc2);
-    }
-    a.device_bc = device_bc ? 1 : 0;
-    a.inv_pre = sa.inv_pre;
-    a.post = sa.post;
 
     cudaError_t e;
     {
@@ -372,8 +382,7 @@ neox_status mt_enqueue(neox_multi* h, float lr, const float* lr_dev, cudaStream_
         if ((e = cudaGetLastError()) != cudaSuccess) return mcuda_fail(h, e, "pass-1 launch");
     }
     if (h->numel > 0) {
-        auto k2 = h->gdtype == NEOX_FP16 ? (h->wdtype == NEOX_FP16 ? mt_adam_kernel<F16, F16> : mt_adam_kernel<F16, BF16>)
-                                         : (h->wdtype == NEOX_FP16 ? mt_adam_kernel<BF16, F16> : mt_adam_kernel<BF16, BF16>);
+        const MtUpdateKernel k2 = mt_update_kernel(h->hp.optimizer == NEOX_SGD, h->gdtype, h->wdtype);
         const int grid = h->grid2;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(grid);
@@ -478,16 +487,19 @@ neox_status neox_multi_create(const neox_tensor_set* set, const neox_hparams* hp
         DevScalars init{};
         init.scale = hp->init_scale;
         init.scale_used = hp->init_scale;
+        init.hyst = hyst_full(*hp);
         if ((e = cudaMemcpy(h->d_sc, &init, sizeof(init), cudaMemcpyHostToDevice)) != cudaSuccess) {
             st = mcuda_fail(nullptr, e, "cudaMemcpy scalars");
             goto done;
         }
         // pass 2 runs with kMtDescBatch3 descriptors of dynamic shared memory
-        auto k2 = h->gdtype == NEOX_FP16 ? (h->wdtype == NEOX_FP16 ? mt_adam_kernel<F16, F16> : mt_adam_kernel<F16, BF16>)
-                                         : (h->wdtype == NEOX_FP16 ? mt_adam_kernel<BF16, F16> : mt_adam_kernel<BF16, BF16>);
+        // (both update rules: set_hparams may switch between them)
+        const MtUpdateKernel k2 = mt_update_kernel(false, h->gdtype, h->wdtype);
+        const MtUpdateKernel k2s = mt_update_kernel(true, h->gdtype, h->wdtype);
         const int dyn = (int)(sizeof(MtTensor) * kMtDescBatch3);
         int occ = 0;
         if ((e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(k2s, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn)) != cudaSuccess ||
             (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k2, kMtThreads3, dyn)) != cudaSuccess) {
             st = mcuda_fail(nullptr, e, "configuring the update kernel");
             goto done;
@@ -611,12 +623,30 @@ neox_status neox_multi_set_state(neox_multi* h, float scale, int32_t good, int64
     s.scale_used = scale;
     s.good = good;
     s.t = t;
+    s.hyst = hyst_full(h->hp);
     if (e == cudaSuccess) e = cudaMemcpy(h->d_sc, &s, sizeof(s), cudaMemcpyHostToDevice);
     if (e != cudaSuccess) return mcuda_fail(h, e, "writing the scaler state");
     h->scale = scale;
     h->good = good;
     h->t = t;
     return NEOX_OK;
+}
+
+neox_status neox_multi_get_hysteresis(const neox_multi* h, int32_t* count) {
+    if (!h || !count) return NEOX_ERR_INVALID_ARGUMENT;
+    DeviceGuard g(h->device);
+    cudaError_t e = h->async_used ? cudaDeviceSynchronize() : cudaSuccess;
+    if (e == cudaSuccess) e = cudaMemcpy(count, &h->d_sc->hyst, sizeof(int32_t), cudaMemcpyDeviceToHost);
+    return e == cudaSuccess ? NEOX_OK : mcuda_fail(const_cast<neox_multi*>(h), e, "reading the hysteresis count");
+}
+
+neox_status neox_multi_set_hysteresis(neox_multi* h, int32_t count) {
+    if (!h) return NEOX_ERR_INVALID_ARGUMENT;
+    if (count < 0) return mfail(h, NEOX_ERR_INVALID_ARGUMENT, "the hysteresis count must be >= 0");
+    DeviceGuard g(h->device);
+    cudaError_t e = h->async_used ? cudaDeviceSynchronize() : cudaSuccess;
+    if (e == cudaSuccess) e = cudaMemcpy(&h->d_sc->hyst, &count, sizeof(int32_t), cudaMemcpyHostToDevice);
+    return e == cudaSuccess ? NEOX_OK : mcuda_fail(h, e, "writing the hysteresis count");
 }
 
 }  // extern "C"

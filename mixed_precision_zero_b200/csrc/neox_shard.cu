@@ -125,14 +125,24 @@ __device__ __forceinline__ void seg_seek(SegCursor& c, unsigned long long i, con
     c.keep = __fsub_rn(1.0f, __fmul_rn(lr, __ldg(seg_wd + lo)));
 }
 
-// The vector loop of pass 2 (KFIX as in pass1_vectors).
-template <class G, class W, int VEC, bool READ_ACC, int KFIX>
+// Store the 16-bit cast of p to every extra destination (indexes fixed at
+// compile time, so the pointer table stays in registers).
+template <class W, int VEC>
+__device__ __forceinline__ void store_copies(const WeightCopies& wc, unsigned long long i, const float (&p)[VEC]) {
+#pragma unroll
+    for (int d = 0; d < kMaxWeightCopies; d++)
+        if (d < wc.n) st16<W, VEC>(wc.p[d] + i, p);
+}
+
+// The vector loop of pass 2 (KFIX as in pass1_vectors).  SGD: plain SGD,
+// which neither reads nor writes m and v; else AdamW.
+template <bool SGD, class G, class W, int VEC, bool READ_ACC, int KFIX, bool COPIES>
 __device__ __forceinline__ void pass2_vectors(const GradPtrs& gp, int K_rt, const float* __restrict__ acc,
                                               const Layout& L, const AdamArgs& a, float c, float inv_us,
                                               float* __restrict__ master, float* __restrict__ m,
                                               float* __restrict__ v, uint16_t* __restrict__ w,
                                               const unsigned long long* __restrict__ seg_end,
-                                              const float* __restrict__ seg_wd, int nsegs) {
+                                              const float* __restrict__ seg_wd, int nsegs, const WeightCopies& wc) {
     const int K = KFIX ? KFIX : K_rt;
     const unsigned long long stride = (unsigned long long)gridDim.x * kThreads3;
     unsigned long long v0 = (unsigned long long)blockIdx.x * kThreads3 + threadIdx.x;
@@ -155,8 +165,10 @@ __device__ __forceinline__ void pass2_vectors(const GradPtrs& gp, int K_rt, cons
             for (int u = 0; u < kUnroll3; u++) {
                 const unsigned long long i = L.head + (vi + u * stride) * VEC;
                 ld32<VEC>(master + i, p[u]);
-                ld32<VEC>(m + i, mm[u]);
-                ld32<VEC>(v + i, vv[u]);
+                if constexpr (!SGD) {
+                    ld32<VEC>(m + i, mm[u]);
+                    ld32<VEC>(v + i, vv[u]);
+                }
             }
 #pragma unroll
             for (int u = 0; u < kUnroll3; u++) {
@@ -173,11 +185,17 @@ __device__ __forceinline__ void pass2_vectors(const GradPtrs& gp, int K_rt, cons
                         keep[e] = cur.keep;
                     }
                 }
-                adam_vec<VEC>(g[u], keep, c, a, p[u], mm[u], vv[u]);
-                st32<VEC>(master + i, p[u]);
-                st32<VEC>(m + i, mm[u]);
-                st32<VEC>(v + i, vv[u]);
+                if constexpr (SGD) {
+                    sgd_vec<VEC>(g[u], keep, c, a.lr, p[u]);
+                    st32<VEC>(master + i, p[u]);
+                } else {
+                    adam_vec<VEC>(g[u], keep, c, a, p[u], mm[u], vv[u]);
+                    st32<VEC>(master + i, p[u]);
+                    st32<VEC>(m + i, mm[u]);
+                    st32<VEC>(v + i, vv[u]);
+                }
                 st16<W, VEC>(w + i, p[u]);
+                if constexpr (COPIES) store_copies<W, VEC>(wc, i, p[u]);
             }
         }
     }
@@ -187,8 +205,10 @@ __device__ __forceinline__ void pass2_vectors(const GradPtrs& gp, int K_rt, cons
         if constexpr (READ_ACC) ld32<VEC>(acc + i, g);
         else ingest<G, VEC>(gp, K, i, a.inv_pre, inv_us, g);
         ld32<VEC>(master + i, p);
-        ld32<VEC>(m + i, mm);
-        ld32<VEC>(v + i, vv);
+        if constexpr (!SGD) {
+            ld32<VEC>(m + i, mm);
+            ld32<VEC>(v + i, vv);
+        }
         if (i >= cur.end) seg_seek(cur, i, seg_end, seg_wd, nsegs, a.lr);
         if (i + VEC <= cur.end) {
 #pragma unroll
@@ -200,20 +220,29 @@ __device__ __forceinline__ void pass2_vectors(const GradPtrs& gp, int K_rt, cons
                 keep[e] = cur.keep;
             }
         }
-        adam_vec<VEC>(g, keep, c, a, p, mm, vv);
-        st32<VEC>(master + i, p);
-        st32<VEC>(m + i, mm);
-        st32<VEC>(v + i, vv);
+        if constexpr (SGD) {
+            sgd_vec<VEC>(g, keep, c, a.lr, p);
+            st32<VEC>(master + i, p);
+        } else {
+            adam_vec<VEC>(g, keep, c, a, p, mm, vv);
+            st32<VEC>(master + i, p);
+            st32<VEC>(m + i, mm);
+            st32<VEC>(v + i, vv);
+        }
         st16<W, VEC>(w + i, p);
+        if constexpr (COPIES) store_copies<W, VEC>(wc, i, p);
     }
 }
 
-template <class G, class W, int VEC, bool READ_ACC>
-__global__ void __launch_bounds__(kThreads3)
-adam_kernel(GradPtrs gp, int K, const float* __restrict__ acc, Layout L, AdamArgs a_arg,
-            float* __restrict__ master, float* __restrict__ m, float* __restrict__ v, uint16_t* __restrict__ w,
-            const unsigned long long* __restrict__ seg_end, const float* __restrict__ seg_wd, int nsegs,
-            const DevScalars* __restrict__ sc) {
+// The whole of pass 2 for one grid: the vector loop, then (block 0) the
+// peeled head and the ragged tail one element per thread.
+template <bool SGD, class G, class W, int VEC, bool READ_ACC, bool COPIES>
+__device__ __forceinline__ void update_shard(const GradPtrs& gp, int K, const float* __restrict__ acc,
+                                             const Layout& L, const AdamArgs& a_arg, float* __restrict__ master,
+                                             float* __restrict__ m, float* __restrict__ v, uint16_t* __restrict__ w,
+                                             const unsigned long long* __restrict__ seg_end,
+                                             const float* __restrict__ seg_wd, int nsegs,
+                                             const DevScalars* __restrict__ sc, const WeightCopies& wc) {
     // Programmatic dependent launch: everything below reads what pass 1 wrote.
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (sc->overflow) return;  // skipped step: nothing is written
@@ -227,26 +256,54 @@ adam_kernel(GradPtrs gp, int K, const float* __restrict__ acc, Layout L, AdamArg
     }
 
     if (K == 1)
-        pass2_vectors<G, W, VEC, READ_ACC, 1>(gp, K, acc, L, a, c, inv_us, master, m, v, w, seg_end, seg_wd, nsegs);
+        pass2_vectors<SGD, G, W, VEC, READ_ACC, 1, COPIES>(gp, K, acc, L, a, c, inv_us, master, m, v, w, seg_end, seg_wd,
+                                                           nsegs, wc);
     else
-        pass2_vectors<G, W, VEC, READ_ACC, 0>(gp, K, acc, L, a, c, inv_us, master, m, v, w, seg_end, seg_wd, nsegs);
+        pass2_vectors<SGD, G, W, VEC, READ_ACC, 0, COPIES>(gp, K, acc, L, a, c, inv_us, master, m, v, w, seg_end, seg_wd,
+                                                           nsegs, wc);
     if (blockIdx.x == 0) {
         const unsigned long long extra = L.head + (L.n - L.tail0);
         for (unsigned long long j = threadIdx.x; j < extra; j += kThreads3) {
             const unsigned long long i = j < L.head ? j : L.tail0 + (j - L.head);
-            float g[1], p[1] = {master[i]}, mm[1] = {m[i]}, vv[1] = {v[i]}, keep[1];
+            float g[1], p[1] = {master[i]}, keep[1];
             if constexpr (READ_ACC) g[0] = acc[i];
             else ingest<G, 1>(gp, K, i, a.inv_pre, inv_us, g);
             SegCursor c1{0, 0ull, 1.0f};
             seg_seek(c1, i, seg_end, seg_wd, nsegs, a.lr);
             keep[0] = c1.keep;
-            adam_vec<1>(g, keep, c, a, p, mm, vv);
+            if constexpr (SGD) {
+                sgd_vec<1>(g, keep, c, a.lr, p);
+            } else {
+                float mm[1] = {m[i]}, vv[1] = {v[i]};
+                adam_vec<1>(g, keep, c, a, p, mm, vv);
+                m[i] = mm[0];
+                v[i] = vv[0];
+            }
             master[i] = p[0];
-            m[i] = mm[0];
-            v[i] = vv[0];
             w[i] = W::enc(p[0]);
+            if constexpr (COPIES) store_copies<W, 1>(wc, i, p);
         }
     }
+}
+
+// Pass 2 with AdamW.
+template <class G, class W, int VEC, bool READ_ACC, bool COPIES>
+__global__ void __launch_bounds__(kThreads3)
+adam_kernel(GradPtrs gp, int K, const float* __restrict__ acc, Layout L, AdamArgs a,
+            float* __restrict__ master, float* __restrict__ m, float* __restrict__ v, uint16_t* __restrict__ w,
+            const unsigned long long* __restrict__ seg_end, const float* __restrict__ seg_wd, int nsegs,
+            const DevScalars* __restrict__ sc, WeightCopies wc) {
+    update_shard<false, G, W, VEC, READ_ACC, COPIES>(gp, K, acc, L, a, master, m, v, w, seg_end, seg_wd, nsegs, sc, wc);
+}
+
+// Pass 2 with plain SGD (m and v are not touched).
+template <class G, class W, int VEC, bool READ_ACC, bool COPIES>
+__global__ void __launch_bounds__(kThreads3)
+sgd_kernel(GradPtrs gp, int K, const float* __restrict__ acc, Layout L, AdamArgs a,
+           float* __restrict__ master, float* __restrict__ m, float* __restrict__ v, uint16_t* __restrict__ w,
+           const unsigned long long* __restrict__ seg_end, const float* __restrict__ seg_wd, int nsegs,
+           const DevScalars* __restrict__ sc, WeightCopies wc) {
+    update_shard<true, G, W, VEC, READ_ACC, COPIES>(gp, K, acc, L, a, master, m, v, w, seg_end, seg_wd, nsegs, sc, wc);
 }
 
 }  // namespace
@@ -281,6 +338,7 @@ struct neox_shard {
     // profiling
     bool profiling = false;
     bool async_used = false;          // an asynchronous step was issued (replays may follow)
+    WeightCopies wcopies{};           // extra destinations of the working weights
     cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};
     neox_profile prof{};
     std::string last_error;
@@ -312,7 +370,9 @@ cudaError_t launch_pass1(neox_shard* h, const GradPtrs& gp, int K, const Layout&
 template <class G, class W, int VEC, bool ACC>
 cudaError_t launch_pass2(neox_shard* h, const GradPtrs& gp, int K, const float* acc, const Layout& L,
                          const AdamArgs& a, uint16_t* w, cudaStream_t st) {
-    auto kern = adam_kernel<G, W, VEC, ACC>;
+    const bool sgd = h->hp.optimizer == NEOX_SGD, copies = h->wcopies.n > 0;
+    auto kern = sgd ? (copies ? sgd_kernel<G, W, VEC, ACC, true> : sgd_kernel<G, W, VEC, ACC, false>)
+                    : (copies ? adam_kernel<G, W, VEC, ACC, true> : adam_kernel<G, W, VEC, ACC, false>);
     const int grid = grid_for(kern, kThreads3, L.nvec, h->sm_count, 1 << 20);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
@@ -328,7 +388,8 @@ cudaError_t launch_pass2(neox_shard* h, const GradPtrs& gp, int K, const float* 
     const unsigned long long* se = h->d_seg_end;
     const float* sw = h->d_seg_wd;
     const DevScalars* sc = h->d_sc;
-    return cudaLaunchKernelEx(&cfg, kern, gp, K, accp, L, a, h->master, h->m, h->v, w, se, sw, h->nsegs, sc);
+    return cudaLaunchKernelEx(&cfg, kern, gp, K, accp, L, a, h->master, h->m, h->v, w, se, sw, h->nsegs, sc,
+                              h->wcopies);
 }
 
 template <class G, int VEC>
@@ -411,7 +472,7 @@ neox_status enqueue_step(neox_shard* h, const void* const* grads, int32_t num_gr
     if (!grads) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "grads is NULL");
     if (!lr_dev && (!finite(lr) || lr < 0.0f)) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "lr must be finite and >= 0");
     GradPtrs gp{};
-    uintptr_t a16[kMaxGrads + 1];
+    uintptr_t a16[kMaxGrads + 1 + kMaxWeightCopies];
     if (h->numel > 0) {
         if (!params) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "params is NULL");
         if ((uintptr_t)params & 1u) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "params must be 2-byte aligned");
@@ -423,6 +484,7 @@ neox_status enqueue_step(neox_shard* h, const void* const* grads, int32_t num_gr
             a16[k] = (uintptr_t)grads[k];
         }
         a16[num_grads] = (uintptr_t)params;
+        for (int d = 0; d < h->wcopies.n; d++) a16[num_grads + 1 + d] = (uintptr_t)h->wcopies.p[d];
     }
     if (result && ((uintptr_t)result & 7u)) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "result must be 8-byte aligned");
     if (mode != kFused && (!stats || ((uintptr_t)stats & 7u)))
@@ -432,45 +494,20 @@ neox_status enqueue_step(neox_shard* h, const void* const* grads, int32_t num_gr
     const bool use_acc = num_grads >= 5 && h->d_acc != nullptr;
     uintptr_t a32[3] = {(uintptr_t)h->master, (uintptr_t)h->m, (uintptr_t)h->v};
     int vec = 1;
-    Layout L = h->numel > 0 ? choose_layout(h->numel, a16, num_grads + 1, a32, 3, vec) : Layout{0, 0, 0, 0};
+    Layout L = h->numel > 0 ? choose_layout(h->numel, a16, num_grads + 1 + h->wcopies.n, a32, 3, vec)
+                            : Layout{0, 0, 0, 0};
     float* acc = nullptr;
     if (use_acc) {
         const unsigned long long hh = L.head % 32;
         acc = h->d_acc + ((32 - hh) % 32);  // &acc[head] sits on a 128-byte line
     }
 
-    ScalerArgs sa{};
-    sa.post = (double)num_grads / (double)h->hp.predivide;
-    sa.inv_pre = (float)(1.0 / (double)h->hp.predivide);
-    sa.clip = h->hp.clip_norm;
-    sa.factor = h->hp.scale_factor;
-    sa.min_scale = h->hp.min_scale;
-    sa.window = h->hp.scale_window;
-    sa.device_bc = device_bc ? 1 : 0;
-    sa.lr = lr;
-    sa.beta1 = h->hp.beta1;
-    sa.beta2 = h->hp.beta2;
+    ScalerArgs sa;
+    AdamArgs a;
+    make_step_args(h->hp, num_grads, lr, h->t, device_bc, sa, a);
     sa.lr_ptr = lr_dev;
     sa.result = result;
     sa.stats_out = mode == kStatsOnly ? stats : nullptr;
-
-    AdamArgs a{};
-    a.lr = lr;
-    a.b1 = h->hp.beta1;
-    a.b2 = h->hp.beta2;
-    a.omb1 = 1.0f - h->hp.beta1;
-    a.omb2 = 1.0f - h->hp.beta2;
-    a.eps = h->hp.eps;
-    if (!device_bc) {
-        const double t1 = (double)(h->t + 1);  // the step count if this step is applied
-        const double bc1 = 1.0 - std::pow((double)h->hp.beta1, t1);
-        const double bc2 = 1.0 - std::pow((double)h->hp.beta2, t1);
-        a.step_size = (float)((double)lr / bc1);
-        a.bcs = (float)std::sqrt(bc2);
-    }
-    a.device_bc = device_bc ? 1 : 0;
-    a.inv_pre = sa.inv_pre;
-    a.post = sa.post;
 
     cudaError_t e;
     if (timed && (e = cudaEventRecord(h->ev[0], st)) != cudaSuccess) return cuda_fail(h, e, "cudaEventRecord");
@@ -657,6 +694,7 @@ neox_status neox_shard_create(const neox_shard_desc* d, const neox_hparams* hp, 
         DevScalars init{};
         init.scale = hp->init_scale;
         init.scale_used = hp->init_scale;
+        init.hyst = hyst_full(*hp);
         if ((e = cudaMemcpy(h->d_sc, &init, sizeof(init), cudaMemcpyHostToDevice)) != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMemcpy scalars"); goto done; }
     }
 done:
@@ -688,6 +726,21 @@ neox_status neox_shard_set_hparams(neox_shard* h, const neox_hparams* hp) {
     return NEOX_OK;
 }
 
+neox_status neox_shard_set_weight_copies(neox_shard* h, void* const* dsts, int32_t n) {
+    if (!h) return NEOX_ERR_INVALID_ARGUMENT;
+    if (n < 0 || n > kMaxWeightCopies) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "n must be in [0, 8]");
+    if (n > 0 && !dsts) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "dsts is NULL");
+    WeightCopies wc{};
+    for (int d = 0; d < n; d++) {
+        if (!dsts[d] || ((uintptr_t)dsts[d] & 1u))
+            return fail(h, NEOX_ERR_INVALID_ARGUMENT, "weight copy " + std::to_string(d) + " NULL or not 2-byte aligned");
+        wc.p[d] = static_cast<uint16_t*>(dsts[d]);
+    }
+    wc.n = n;
+    h->wcopies = wc;
+    return NEOX_OK;
+}
+
 neox_status neox_shard_get_state(const neox_shard* h, float* scale, int32_t* good, int64_t* t) {
     if (!h) return NEOX_ERR_INVALID_ARGUMENT;
     if (neox_status s = refresh_mirror(const_cast<neox_shard*>(h)); s != NEOX_OK) return s;
@@ -711,12 +764,31 @@ neox_status neox_shard_set_state(neox_shard* h, float scale, int32_t good, int64
     s.scale_used = scale;
     s.good = good;
     s.t = t;
+    s.hyst = hyst_full(h->hp);
     cudaError_t e = cudaMemcpy(h->d_sc, &s, sizeof(s), cudaMemcpyHostToDevice);
     if (e != cudaSuccess) return cuda_fail(h, e, "cudaMemcpy scalars");
     h->scale = scale;
     h->good = good;
     h->t = t;
     return NEOX_OK;
+}
+
+neox_status neox_shard_get_hysteresis(const neox_shard* h, int32_t* count) {
+    if (!h || !count) return NEOX_ERR_INVALID_ARGUMENT;
+    auto* hm = const_cast<neox_shard*>(h);
+    DeviceGuard g(h->device);
+    cudaError_t e = h->async_used ? cudaDeviceSynchronize() : cudaSuccess;
+    if (e == cudaSuccess) e = cudaMemcpy(count, &h->d_sc->hyst, sizeof(int32_t), cudaMemcpyDeviceToHost);
+    return e == cudaSuccess ? NEOX_OK : cuda_fail(hm, e, "reading the hysteresis count");
+}
+
+neox_status neox_shard_set_hysteresis(neox_shard* h, int32_t count) {
+    if (!h) return NEOX_ERR_INVALID_ARGUMENT;
+    if (count < 0) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "the hysteresis count must be >= 0");
+    DeviceGuard g(h->device);
+    cudaError_t e = h->async_used ? cudaDeviceSynchronize() : cudaSuccess;
+    if (e == cudaSuccess) e = cudaMemcpy(&h->d_sc->hyst, &count, sizeof(int32_t), cudaMemcpyHostToDevice);
+    return e == cudaSuccess ? NEOX_OK : cuda_fail(h, e, "writing the hysteresis count");
 }
 
 neox_status neox_shard_set_profiling(neox_shard* h, int32_t enable) {
@@ -879,6 +951,9 @@ neox_status neox_shard_step_noalloc(const neox_shard_desc* d, const neox_hparams
         snprintf(g_noalloc_error, sizeof(g_noalloc_error), "%s", why);
         return NEOX_ERR_INVALID_ARGUMENT;
     }
+    if (hp->hysteresis > 1)
+        return noalloc_fail(NEOX_ERR_INVALID_ARGUMENT, "hysteresis %lld needs a handle (neox_shard_create): the "
+                            "scaler state of this call has no hysteresis count", hp->hysteresis);
     if ((d->wdtype != NEOX_FP16 && d->wdtype != NEOX_BF16) || (d->gdtype != NEOX_FP16 && d->gdtype != NEOX_BF16))
         return noalloc_fail(NEOX_ERR_INVALID_ARGUMENT, "dtype must be NEOX_FP16 or NEOX_BF16");
     if (!(state->scale > 0.0f) || !finite(state->scale) || state->good < 0 || state->t < 0)
@@ -941,6 +1016,7 @@ neox_status neox_shard_step_noalloc(const neox_shard_desc* d, const neox_hparams
     v.sm_count = nd->sm_count;
     v.max_parts = nd->sm_count * kMaxBlocksPerSm < kNoallocMaxParts ? nd->sm_count * kMaxBlocksPerSm : kNoallocMaxParts;
     v.numel = d->numel;
+    v.hp = *hp;
     v.master = d->master;
     v.m = d->exp_avg;
     v.v = d->exp_avg_sq;
@@ -958,6 +1034,7 @@ neox_status neox_shard_step_noalloc(const neox_shard_desc* d, const neox_hparams
     init.scale_used = state->scale;
     init.good = state->good;
     init.t = state->t;
+    init.hyst = 1;
     if ((e = cudaMemcpyAsync(v.d_sc, &init, sizeof(init), cudaMemcpyHostToDevice, st)) != cudaSuccess ||
         (e = cudaMemcpyAsync(v.d_seg_end, ends, sizeof(unsigned long long) * nsegs, cudaMemcpyHostToDevice, st)) != cudaSuccess ||
         (e = cudaMemcpyAsync(v.d_seg_wd, wds, sizeof(float) * nsegs, cudaMemcpyHostToDevice, st)) != cudaSuccess)
@@ -967,29 +1044,9 @@ neox_status neox_shard_step_noalloc(const neox_shard_desc* d, const neox_hparams
     int vec = 1;
     Layout L = d->numel > 0 ? choose_layout(d->numel, a16, num_grads + 1, a32, 3, vec) : Layout{0, 0, 0, 0};
 
-    ScalerArgs sa{};
-    sa.post = (double)num_grads / (double)hp->predivide;
-    sa.inv_pre = (float)(1.0 / (double)hp->predivide);
-    sa.clip = hp->clip_norm;
-    sa.factor = hp->scale_factor;
-    sa.min_scale = hp->min_scale;
-    sa.window = hp->scale_window;
-    AdamArgs a{};
-    a.lr = lr;
-    a.b1 = hp->beta1;
-    a.b2 = hp->beta2;
-    a.omb1 = 1.0f - hp->beta1;
-    a.omb2 = 1.0f - hp->beta2;
-    a.eps = hp->eps;
-    {
-        const double t1 = (double)(state->t + 1);
-        const double bc1 = 1.0 - std::pow((double)hp->beta1, t1);
-        const double bc2 = 1.0 - std::pow((double)hp->beta2, t1);
-        a.step_size = (float)((double)lr / bc1);
-        a.bcs = (float)std::sqrt(bc2);
-    }
-    a.inv_pre = sa.inv_pre;
-    a.post = sa.post;
+    ScalerArgs sa;
+    AdamArgs a;
+    make_step_args(*hp, num_grads, lr, state->t, false, sa, a);
 
     // K >= 5 re-reads the K buffers in pass 2 (no FP32-sum buffer: it would
     // need numel * 4 bytes of scratch).

@@ -57,6 +57,13 @@ def ordered16(h: np.ndarray) -> np.ndarray:
     return np.where(h & 0x8000, -(h & 0x7FFF), h)
 
 
+def oracle_hparams(hp: Hparams):
+    """The oracle's copy of the library's hyperparameters."""
+    return oracle.OracleHparams(hp.beta1, hp.beta2, hp.eps, hp.clip_norm, hp.predivide, hp.init_scale,
+                                hp.scale_factor, hp.min_scale, hp.scale_window, hysteresis=hp.hysteresis,
+                                optimizer={"adamw": 0, "sgd": 1}[hp.optimizer])
+
+
 class ShardCase:
     """A shard on the GPU (driven through the C ABI) and the oracle's copy."""
 
@@ -88,9 +95,7 @@ class ShardCase:
         self.shard = NeoxShard(self.master.t, self.m.t, self.v.t, self.hp,
                                wdtype=_torch_dtype(wbf16), gdtype=_torch_dtype(gbf16),
                                segments=segments, weight_decay=default_wd, max_grads=max_grads)
-        ohp = oracle.OracleHparams(self.hp.beta1, self.hp.beta2, self.hp.eps, self.hp.clip_norm,
-                                   self.hp.predivide, self.hp.init_scale, self.hp.scale_factor,
-                                   self.hp.min_scale, self.hp.scale_window)
+        ohp = oracle_hparams(self.hp)
         master_host = self.master.t.cpu().numpy()
         self.orc = oracle.OracleShard(master_host, ohp, wbf16=wbf16, gbf16=gbf16, segments=segments,
                                       default_wd=default_wd)

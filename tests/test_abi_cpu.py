@@ -78,6 +78,8 @@ def _hp(**kw):
     ({}, {"scale_factor": 0.5}, "scale_factor"),
     ({}, {"min_scale": -1.0}, "min_scale"),
     ({}, {"scale_window": 0}, "scale_window"),
+    ({}, {"hysteresis": -1}, "hysteresis"),
+    ({}, {"optimizer": 2}, "optimizer"),
     ({"wdtype": 7}, {}, "dtype"),
     ({"master": 0}, {}, "non-NULL"),
     ({"exp_avg": 8194}, {}, "aligned"),

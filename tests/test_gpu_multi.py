@@ -10,7 +10,7 @@ import torch
 import oracle
 import synth
 from mixed_precision_zero_b200 import Hparams, NeoxError, NeoxMultiShard, NeoxShard, _abi
-from tests.gpu_harness import Guarded, check_close, check_ulp16, to_u16
+from tests.gpu_harness import Guarded, check_close, check_ulp16, oracle_hparams, to_u16
 
 pytestmark = pytest.mark.gpu
 
@@ -47,8 +47,7 @@ class MultiCase:
             off += p["n"]
         self.total = off
         master = np.concatenate([p["master"].t.cpu().numpy() for p in self.parts])
-        ohp = oracle.OracleHparams(self.hp.beta1, self.hp.beta2, self.hp.eps, self.hp.clip_norm, self.hp.predivide,
-                                   self.hp.init_scale, self.hp.scale_factor, self.hp.min_scale, self.hp.scale_window)
+        ohp = oracle_hparams(self.hp)
         self.orc = oracle.OracleShard(master, ohp, wbf16=wbf16, gbf16=gbf16, segments=segs)
 
     def gen(self, s, sigma):

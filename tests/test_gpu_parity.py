@@ -328,3 +328,33 @@ def test_maximum_buffer_count(max_grads):
         c.check_state()
     assert c.guards_intact()
     c.close()
+
+
+@pytest.mark.parametrize("offsets", [[0, 0, 0], [3, 3, 3], [1, 2, 0]])
+def test_weight_copies_receive_the_cast(offsets):
+    """Pass 2 writes the updated 16-bit weights into every registered copy
+    (the all-gather destinations of the other ranks, here local buffers at
+    chosen element offsets), byte-identical to params, and leaves them alone
+    on a skipped step."""
+    n = 250_003
+    c = ShardCase(n, hp=Hparams(init_scale=2.0 ** 12, scale_window=3), offsets={"all": offsets[0]}, lr=1e-3)
+    copies = [Guarded(n, torch.float16, o) for o in offsets]
+    for x in copies:
+        x.t.fill_(0.0)
+    c.shard.set_weight_copies([x.t for x in copies])
+    for s in range(1, 5):
+        c.gen_normal(s, 1e-3)
+        if s == 3:
+            c.inject(s)
+            before = [x.t.clone() for x in copies]
+        res, info = c.step()
+        c.check_result(res, info)
+        c.check_state()
+        for j, x in enumerate(copies):
+            if s == 3:
+                assert torch.equal(x.t.view(torch.int16), before[j].view(torch.int16))
+            else:
+                assert torch.equal(x.t.view(torch.int16), c.w.t.view(torch.int16))
+            assert x.guards_intact()
+    c.shard.set_weight_copies([])
+    c.close()
