@@ -387,6 +387,7 @@ def run_b200(args):
     import torch
     import torch.distributed as dist
 
+    from mixed_precision_zero_b200.zero import zero_step
     from synth import workloads as W
     ws, rank, local = dist_env()
     if ws != args.gpus:
@@ -414,9 +415,9 @@ def run_b200(args):
     def one_step():
         if not split:
             return shard.step(grads, params, wl.lr)
-        shard.grad_stats(grads, params, stats)
         if dist.is_initialized():
-            dist.all_reduce(stats)
+            return zero_step(shard, grads, params, wl.lr, stats)
+        shard.grad_stats(grads, params, stats)
         return shard.apply(grads, params, wl.lr, stats)
 
     for _ in range(args.warmup):

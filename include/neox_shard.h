@@ -108,7 +108,14 @@ typedef struct {
                                      K >= 5 makes create reserve numel*4 bytes
                                      of FP32 scratch so pass 2 reads one FP32
                                      sum instead of re-reading K buffers       */
+    int32_t flags;                /* 0 or NEOX_SHARD_ACCUMULATE                */
 } neox_shard_desc;
+
+/* neox_shard_desc.flags: reserve the FP32 sum buffer whatever max_grads is,
+ * and use it at every K: pass 1 writes the FP32 sum of the K buffers, pass 2
+ * reads it instead of re-reading them.  Meant for gradient buffers in peer
+ * memory (the ZeRO-2 form below), which pass 1 then reads over NVLink once. */
+#define NEOX_SHARD_ACCUMULATE 1
 
 typedef struct {
     int32_t overflow;          /* 1: non-finite gradient; the step was skipped */
@@ -223,6 +230,48 @@ neox_status neox_shard_apply(neox_shard* h, const void* const* grads, int32_t nu
  * them into account (a destination with another residue mod 16 bytes makes
  * the kernels use narrower vectors). */
 neox_status neox_shard_set_weight_copies(neox_shard* h, void* const* dsts, int32_t n);
+
+/* ------------------------------------------------------------------------
+ * ZeRO-2: the gradient reduce-scatter fused with pass 1, through CUDA IPC.
+ *
+ * Under ZeRO stage 2 every rank holds the full gradient of its own
+ * micro-batches, and the owner of each flat slice needs the sum over the
+ * ranks of that slice ("GPT-NeoX: how it opened the door to democratised
+ * 100B-scale training" (ainews.cool), "技术深度解析": DP + ZeRO pairs with
+ * reduce-scatter / all-gather; the OPT summary, "方法适配": the pre-divide is
+ * applied before that cross-rank sum).  The step's K-buffer ingest is that
+ * sum: pass neox_shard_step (or grad_stats / apply) the K = world-size
+ * pointers peer_j + rank * slice_bytes, one per rank j, where peer_j is rank
+ * j's full gradient buffer mapped into this process (neox_ipc_open; this
+ * rank's own buffer directly).  Pass 1 then reads every rank's copy of this
+ * rank's slice straight from its owner's HBM over NVLink, pre-divides, sums
+ * in FP32 in rank order and reduces the norm, with no reduce-scatter
+ * collective and no staging copy; with NEOX_SHARD_ACCUMULATE the FP32 sum
+ * stays in local memory for pass 2.  The split step's 16-byte all-reduce
+ * then gives every rank the same decision, and neox_shard_set_weight_copies
+ * pointed at the peers' full-weight buffers performs the all-gather.
+ *
+ * The calls below wrap CUDA IPC (one node; handles are plain bytes that the
+ * caller exchanges, e.g. with torch.distributed).  Errors: NEOX_ERR_CUDA
+ * (message in neox_ipc_last_error(), per thread) or
+ * NEOX_ERR_INVALID_ARGUMENT for NULL arguments.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    unsigned char bytes[64];   /* a cudaIpcMemHandle_t, opaque */
+} neox_ipc_handle;
+
+/* Export the device allocation that contains dev_ptr: *handle names the whole
+ * allocation (cudaMalloc'd memory; not stream-ordered or virtual-memory
+ * allocations), *offset is dev_ptr's byte offset inside it. */
+neox_status neox_ipc_export(const void* dev_ptr, neox_ipc_handle* handle, uint64_t* offset);
+/* Map an allocation another process exported into this process's current
+ * device (peer access enabled lazily); *base is its start: add the
+ * exporter's offset.  A process cannot open a handle it exported itself, and
+ * opens each handle once (share the mapping).  Close before the exporter
+ * frees the memory. */
+neox_status neox_ipc_open(const neox_ipc_handle* handle, void** base);
+neox_status neox_ipc_close(void* base);
+const char* neox_ipc_last_error(void);
 
 /* Replace the hyperparameters (e.g. the clip 1.0 -> 0.3 change, or a switch
  * to NEOX_SGD); the current loss scale and counters are kept (init_scale is
@@ -356,7 +405,8 @@ const char* neox_multi_last_error(const neox_multi* h);
  * Limits: at most 1024 segments (a longer table is rejected with
  * NEOX_ERR_INVALID_ARGUMENT and a message); K in [1, 64].  There is no FP32
  * gradient-sum buffer (it would need numel*4 bytes), so K >= 5 re-reads the K
- * buffers in pass 2; desc->max_grads is ignored.  numel itself is not limited.
+ * buffers in pass 2; desc->max_grads and desc->flags are ignored.  numel itself
+ * is not limited.
  * The scaler state below has no hysteresis count, so hp->hysteresis must be
  * 0 or 1 (a larger value is rejected); hp->optimizer is honoured.
  *

@@ -26,7 +26,8 @@ from ._abi import (NEOX_BF16, NEOX_ERR_CUDA, NEOX_ERR_INVALID_ARGUMENT, NEOX_ERR
                    neox_multi_rebind_grads, neox_multi_get_state, neox_multi_set_state,
                    neox_multi_set_hparams, neox_multi_destroy, neox_shard_grad_stats, neox_shard_apply,
                    neox_shard_set_weight_copies, neox_shard_get_hysteresis, neox_shard_set_hysteresis,
-                   neox_multi_get_hysteresis, neox_multi_set_hysteresis, NEOX_ADAMW, NEOX_SGD)
+                   neox_multi_get_hysteresis, neox_multi_set_hysteresis, NEOX_ADAMW, NEOX_SGD,
+                   NEOX_SHARD_ACCUMULATE)
 
 __all__ = ["NeoxShard", "NeoxMultiShard", "Hparams", "NeoxError", "neox_shard_create", "neox_shard_step",
            "neox_shard_destroy", "neox_shard_set_hparams", "neox_shard_get_state",
@@ -56,6 +57,10 @@ class Hparams:
                             self.hysteresis, opts[self.optimizer])
 
 
+def _ptr(g) -> int:
+    return g if isinstance(g, int) else g.data_ptr()
+
+
 def _dtype_code(t) -> int:
     import torch
     if t.dtype == torch.float16:
@@ -71,7 +76,7 @@ class NeoxShard:
 
     def __init__(self, master, exp_avg, exp_avg_sq, hp: Hparams | None = None, *,
                  wdtype=None, gdtype=None, segments=None, weight_decay: float = 0.0,
-                 max_grads: int = 1, device: int | None = None):
+                 max_grads: int = 1, device: int | None = None, accumulate: bool = False):
         import torch
         hp = hp or Hparams()
         n = master.numel()
@@ -90,7 +95,8 @@ class NeoxShard:
             self._segs, segp, nsegs = None, None, 0
         desc = neox_shard_desc(n, self.wdtype, self.gdtype, segp, nsegs, float(weight_decay),
                                master.data_ptr() if n else None, exp_avg.data_ptr() if n else None,
-                               exp_avg_sq.data_ptr() if n else None, int(max_grads))
+                               exp_avg_sq.data_ptr() if n else None, int(max_grads),
+                               NEOX_SHARD_ACCUMULATE if accumulate else 0)
         self.device = master.device.index if device is None else device
         if self.device is None:
             self.device = torch.cuda.current_device()
@@ -98,6 +104,8 @@ class NeoxShard:
 
     def _check(self, grads, params):
         for g in grads:
+            if isinstance(g, int):   # a raw device pointer (e.g. a peer's slice), the caller's to size
+                continue
             if g.numel() != self.numel or _dtype_code(g) != self.gdtype or not g.is_contiguous():
                 raise ValueError("each grad must be a contiguous 16-bit tensor of the shard's gradient type and length")
         if params.numel() != self.numel or _dtype_code(params) != self.wdtype or not params.is_contiguous():
@@ -109,7 +117,7 @@ class NeoxShard:
         if stream is None:
             stream = torch.cuda.current_stream(self.device)
         sp = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
-        return neox_shard_step(self.handle, [g.data_ptr() for g in grads], params.data_ptr(), lr, sp)
+        return neox_shard_step(self.handle, [_ptr(g) for g in grads], params.data_ptr(), lr, sp)
 
     def step_async(self, grads, params, lr: float = 0.0, *, result=None, lr_device=None, stream=None) -> None:
         """Enqueue a step without waiting.  `result`: a device (or pinned) tensor
@@ -120,7 +128,7 @@ class NeoxShard:
         if stream is None:
             stream = torch.cuda.current_stream(self.device)
         sp = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
-        neox_shard_step_async(self.handle, [g.data_ptr() for g in grads], params.data_ptr(), lr, sp,
+        neox_shard_step_async(self.handle, [_ptr(g) for g in grads], params.data_ptr(), lr, sp,
                               None if result is None else result.data_ptr(),
                               None if lr_device is None else lr_device.data_ptr())
 
@@ -135,7 +143,7 @@ class NeoxShard:
         if stream is None:
             stream = torch.cuda.current_stream(self.device)
         sp = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
-        neox_shard_grad_stats(self.handle, [g.data_ptr() for g in grads], params.data_ptr(), sp, stats.data_ptr())
+        neox_shard_grad_stats(self.handle, [_ptr(g) for g in grads], params.data_ptr(), sp, stats.data_ptr())
 
     def apply(self, grads, params, lr: float, stats, stream=None) -> neox_step_result:
         """The step's decisions from the (all-reduced) statistics, then pass 2."""
@@ -144,17 +152,20 @@ class NeoxShard:
         if stream is None:
             stream = torch.cuda.current_stream(self.device)
         sp = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
-        return neox_shard_apply(self.handle, [g.data_ptr() for g in grads], params.data_ptr(), lr, stats.data_ptr(), sp)
+        return neox_shard_apply(self.handle, [_ptr(g) for g in grads], params.data_ptr(), lr, stats.data_ptr(), sp)
 
     def set_weight_copies(self, dsts) -> None:
-        """Extra 16-bit tensors (same length and type as params) that pass 2
-        writes with the updated weights, e.g. peer-mapped slices of every
-        rank's full-weight buffer.  An empty list removes them."""
+        """Extra 16-bit tensors (same length and type as params), or raw device
+        pointers to such arrays, that pass 2 writes with the updated weights,
+        e.g. peer-mapped slices of every rank's full-weight buffer
+        (see peer.PeerMap).  An empty list removes them."""
         for d in dsts:
+            if isinstance(d, int):   # a raw device pointer (e.g. a slice of a peer's weight buffer)
+                continue
             if d.numel() != self.numel or _dtype_code(d) != self.wdtype or not d.is_contiguous():
                 raise ValueError("each copy must be a contiguous 16-bit tensor like params")
         self._copies = list(dsts)  # keep them alive
-        neox_shard_set_weight_copies(self.handle, [d.data_ptr() for d in dsts])
+        neox_shard_set_weight_copies(self.handle, [_ptr(d) for d in dsts])
 
     def set_hparams(self, hp: Hparams) -> None:
         neox_shard_set_hparams(self.handle, hp.c())
@@ -170,6 +181,18 @@ class NeoxShard:
 
     def set_hysteresis(self, count: int) -> None:
         neox_shard_set_hysteresis(self.handle, count)
+
+    def state_dict(self) -> dict:
+        """The library-held step state for a checkpoint (master / m / v and the
+        working weights are the caller's tensors and are saved with the model)."""
+        scale, good, t = self.get_state()
+        return {"loss_scale": scale, "good_steps": good, "applied_steps": t,
+                "hysteresis_count": self.get_hysteresis()}
+
+    def load_state_dict(self, d: dict) -> None:
+        """Resume exactly where state_dict() was taken."""
+        self.set_state(d["loss_scale"], d["good_steps"], d["applied_steps"])
+        self.set_hysteresis(d["hysteresis_count"])
 
     def set_profiling(self, enable: bool) -> None:
         neox_shard_set_profiling(self.handle, enable)
@@ -263,6 +286,15 @@ class NeoxMultiShard:
 
     def set_hysteresis(self, count: int) -> None:
         neox_multi_set_hysteresis(self.handle, count)
+
+    def state_dict(self) -> dict:
+        scale, good, t = self.get_state()
+        return {"loss_scale": scale, "good_steps": good, "applied_steps": t,
+                "hysteresis_count": self.get_hysteresis()}
+
+    def load_state_dict(self, d: dict) -> None:
+        self.set_state(d["loss_scale"], d["good_steps"], d["applied_steps"])
+        self.set_hysteresis(d["hysteresis_count"])
 
     def set_hparams(self, hp: Hparams) -> None:
         neox_multi_set_hparams(self.handle, hp.c())

@@ -23,6 +23,8 @@ NEOX_BF16 = 1
 NEOX_ADAMW = 0
 NEOX_SGD = 1
 
+NEOX_SHARD_ACCUMULATE = 1
+
 
 class neox_segment(ctypes.Structure):
     _fields_ = [("offset", ctypes.c_uint64), ("numel", ctypes.c_uint64), ("weight_decay", ctypes.c_float)]
@@ -41,7 +43,7 @@ class neox_shard_desc(ctypes.Structure):
                 ("segs", ctypes.POINTER(neox_segment)), ("nsegs", ctypes.c_int32),
                 ("default_weight_decay", ctypes.c_float),
                 ("master", ctypes.c_void_p), ("exp_avg", ctypes.c_void_p), ("exp_avg_sq", ctypes.c_void_p),
-                ("max_grads", ctypes.c_int32)]
+                ("max_grads", ctypes.c_int32), ("flags", ctypes.c_int32)]
 
 
 class neox_step_result(ctypes.Structure):
@@ -51,6 +53,10 @@ class neox_step_result(ctypes.Structure):
 
     def as_dict(self) -> dict:
         return {k: getattr(self, k) for k, _ in self._fields_}
+
+
+class neox_ipc_handle(ctypes.Structure):
+    _fields_ = [("bytes", ctypes.c_ubyte * 64)]
 
 
 class neox_scaler_state(ctypes.Structure):
@@ -163,6 +169,14 @@ def lib() -> ctypes.CDLL:
         L.neox_multi_last_error.restype = ctypes.c_char_p
         L.neox_noalloc_last_error.argtypes = []
         L.neox_noalloc_last_error.restype = ctypes.c_char_p
+        L.neox_ipc_export.argtypes = [ctypes.c_void_p, ctypes.POINTER(neox_ipc_handle), ctypes.POINTER(ctypes.c_uint64)]
+        L.neox_ipc_export.restype = S
+        L.neox_ipc_open.argtypes = [ctypes.POINTER(neox_ipc_handle), ctypes.POINTER(ctypes.c_void_p)]
+        L.neox_ipc_open.restype = S
+        L.neox_ipc_close.argtypes = [ctypes.c_void_p]
+        L.neox_ipc_close.restype = S
+        L.neox_ipc_last_error.argtypes = []
+        L.neox_ipc_last_error.restype = ctypes.c_char_p
         _lib = L
     return _lib
 
@@ -374,3 +388,33 @@ def neox_shard_set_weight_copies(h: int, dst_ptrs) -> None:
     st = lib().neox_shard_set_weight_copies(h, arr, len(dst_ptrs))
     if st != NEOX_OK:
         raise NeoxError(st, lib().neox_last_error(h).decode())
+
+
+# ---- CUDA IPC (peer buffers for the fused reduce-scatter / all-gather) ---------------
+
+def neox_ipc_export(dev_ptr: int):
+    """(64 handle bytes, byte offset of dev_ptr in the exported allocation)."""
+    h, off = neox_ipc_handle(), ctypes.c_uint64()
+    st = lib().neox_ipc_export(dev_ptr, ctypes.byref(h), ctypes.byref(off))
+    if st != NEOX_OK:
+        raise NeoxError(st, lib().neox_ipc_last_error().decode())
+    return bytes(h.bytes), off.value
+
+
+def neox_ipc_open(handle: bytes) -> int:
+    """Map a peer process's exported allocation; returns its base address."""
+    if len(handle) != 64:
+        raise ValueError("an IPC handle is 64 bytes")
+    h = neox_ipc_handle()
+    ctypes.memmove(h.bytes, handle, 64)
+    base = ctypes.c_void_p()
+    st = lib().neox_ipc_open(ctypes.byref(h), ctypes.byref(base))
+    if st != NEOX_OK:
+        raise NeoxError(st, lib().neox_ipc_last_error().decode())
+    return base.value
+
+
+def neox_ipc_close(base: int) -> None:
+    st = lib().neox_ipc_close(base)
+    if st != NEOX_OK:
+        raise NeoxError(st, lib().neox_ipc_last_error().decode())

@@ -21,7 +21,7 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-shared",
                      "-Xptxas", "-v", "-I", INCLUDE]
 
-SOURCES = [os.path.join(PKG, "csrc", "neox_shard.cu"), os.path.join(PKG, "csrc", "neox_multi.cu")]
+SOURCES = [os.path.join(PKG, "csrc", f) for f in ("neox_shard.cu", "neox_multi.cu", "neox_peer.cu")]
 LIB = os.path.join(PKG, "libneoxshard.so")
 
 

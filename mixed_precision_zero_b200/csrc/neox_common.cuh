@@ -19,7 +19,8 @@ constexpr int kMaxGrads = 64;
 constexpr int kThreads1 = 512;   // pass-1 block
 constexpr int kUnroll1 = 4;      // pass-1 vectors in flight per thread
 constexpr int kThreads3 = 256;   // pass-2 block
-constexpr int kUnroll3 = 1;      // pass-2 vectors in flight per thread
+constexpr int kUnroll3 = 1;      // pass-2 vectors in flight per thread (AdamW)
+constexpr int kUnrollSgd = 4;    // pass-2 vectors in flight per thread (SGD): measured 6.25 TB/s against 5.83 at 1
 constexpr int kMaxBlocksPerSm = 32;
 
 struct GradPtrs {

@@ -144,25 +144,26 @@ __device__ __forceinline__ void pass2_vectors(const GradPtrs& gp, int K_rt, cons
                                               const unsigned long long* __restrict__ seg_end,
                                               const float* __restrict__ seg_wd, int nsegs, const WeightCopies& wc) {
     const int K = KFIX ? KFIX : K_rt;
+    constexpr int U = SGD ? kUnrollSgd : kUnroll3;
     const unsigned long long stride = (unsigned long long)gridDim.x * kThreads3;
     unsigned long long v0 = (unsigned long long)blockIdx.x * kThreads3 + threadIdx.x;
     SegCursor cur{0, 0ull, 1.0f};
     if (v0 < L.nvec) seg_seek(cur, L.head + v0 * VEC, seg_end, seg_wd, nsegs, a.lr);
 
     unsigned long long vi = v0;
-    // kUnroll3 strides per iteration: every load of the batch is issued before
+    // U strides per iteration: every load of the batch is issued before
     // the first update, to keep more bytes in flight per thread.
-    if constexpr (kUnroll3 > 1) {
-        for (; vi + (kUnroll3 - 1) * stride < L.nvec; vi += kUnroll3 * stride) {
-            float g[kUnroll3][VEC], p[kUnroll3][VEC], mm[kUnroll3][VEC], vv[kUnroll3][VEC];
+    if constexpr (U > 1) {
+        for (; vi + (U - 1) * stride < L.nvec; vi += U * stride) {
+            float g[U][VEC], p[U][VEC], mm[U][VEC], vv[U][VEC];
             if constexpr (READ_ACC) {
 #pragma unroll
-                for (int u = 0; u < kUnroll3; u++) ld32<VEC>(acc + L.head + (vi + u * stride) * VEC, g[u]);
+                for (int u = 0; u < U; u++) ld32<VEC>(acc + L.head + (vi + u * stride) * VEC, g[u]);
             } else {
-                ingest_batch<G, VEC, kUnroll3>(gp, K, L.head + vi * VEC, stride * VEC, a.inv_pre, inv_us, g);
+                ingest_batch<G, VEC, U>(gp, K, L.head + vi * VEC, stride * VEC, a.inv_pre, inv_us, g);
             }
 #pragma unroll
-            for (int u = 0; u < kUnroll3; u++) {
+            for (int u = 0; u < U; u++) {
                 const unsigned long long i = L.head + (vi + u * stride) * VEC;
                 ld32<VEC>(master + i, p[u]);
                 if constexpr (!SGD) {
@@ -171,7 +172,7 @@ __device__ __forceinline__ void pass2_vectors(const GradPtrs& gp, int K_rt, cons
                 }
             }
 #pragma unroll
-            for (int u = 0; u < kUnroll3; u++) {
+            for (int u = 0; u < U; u++) {
                 const unsigned long long i = L.head + (vi + u * stride) * VEC;
                 float keep[VEC];
                 if (i >= cur.end) seg_seek(cur, i, seg_end, seg_wd, nsegs, a.lr);
@@ -320,6 +321,7 @@ struct neox_shard {
     float* v = nullptr;
     neox_hparams hp{};
     int max_grads = 1;
+    bool accumulate = false;          // NEOX_SHARD_ACCUMULATE: the FP32 sum buffer at every K
     // mirrors of the device scaler state (refreshed after every step)
     float scale = 1.0f;
     int32_t good = 0;
@@ -491,7 +493,7 @@ neox_status enqueue_step(neox_shard* h, const void* const* grads, int32_t num_gr
         return fail(h, NEOX_ERR_INVALID_ARGUMENT, "stats must be a non-NULL, 8-byte aligned device pointer");
     if (lr_dev && ((uintptr_t)lr_dev & 3u)) return fail(h, NEOX_ERR_INVALID_ARGUMENT, "lr_device must be 4-byte aligned");
 
-    const bool use_acc = num_grads >= 5 && h->d_acc != nullptr;
+    const bool use_acc = h->d_acc != nullptr && (num_grads >= 5 || h->accumulate);
     uintptr_t a32[3] = {(uintptr_t)h->master, (uintptr_t)h->m, (uintptr_t)h->v};
     int vec = 1;
     Layout L = h->numel > 0 ? choose_layout(h->numel, a16, num_grads + 1 + h->wcopies.n, a32, 3, vec)
@@ -602,6 +604,7 @@ neox_status neox_shard_create(const neox_shard_desc* d, const neox_hparams* hp, 
         return fail(nullptr, NEOX_ERR_INVALID_ARGUMENT, "dtype must be NEOX_FP16 or NEOX_BF16");
     if (d->max_grads < 0 || d->max_grads > kMaxGrads)
         return fail(nullptr, NEOX_ERR_INVALID_ARGUMENT, "max_grads must be in [0, 64]");
+    if (d->flags & ~NEOX_SHARD_ACCUMULATE) return fail(nullptr, NEOX_ERR_INVALID_ARGUMENT, "unknown flags");
     if (d->numel > 0) {
         if (!d->master || !d->exp_avg || !d->exp_avg_sq)
             return fail(nullptr, NEOX_ERR_INVALID_ARGUMENT, "master/exp_avg/exp_avg_sq must be non-NULL");
@@ -653,6 +656,7 @@ neox_status neox_shard_create(const neox_shard_desc* d, const neox_hparams* hp, 
     h->v = d->exp_avg_sq;
     h->hp = *hp;
     h->max_grads = d->max_grads < 1 ? 1 : d->max_grads;
+    h->accumulate = (d->flags & NEOX_SHARD_ACCUMULATE) != 0;
     h->scale = hp->init_scale;
     h->nsegs = nsegs;
 
@@ -678,7 +682,7 @@ neox_status neox_shard_create(const neox_shard_desc* d, const neox_hparams* hp, 
         if ((e = cudaMalloc(&h->d_seg_end, sizeof(unsigned long long) * nsegs)) != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMalloc segments"); goto done; }
         if ((e = cudaMalloc(&h->d_seg_wd, sizeof(float) * nsegs)) != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMalloc segments"); goto done; }
         bytes += (sizeof(unsigned long long) + sizeof(float)) * nsegs;
-        if (h->max_grads >= 5 && h->numel > 0) {
+        if ((h->max_grads >= 5 || h->accumulate) && h->numel > 0) {
             if ((e = cudaMalloc(&h->d_acc, sizeof(float) * (h->numel + 32))) != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMalloc accumulation buffer"); goto done; }
             bytes += sizeof(float) * (h->numel + 32);
         }

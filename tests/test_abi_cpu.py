@@ -59,6 +59,7 @@ def _desc(n=16, **kw):
     d.exp_avg_sq = kw.get("exp_avg_sq", 12288)
     d.default_weight_decay = kw.get("wd", 0.1)
     d.max_grads = kw.get("max_grads", 1)
+    d.flags = kw.get("flags", 0)
     return d
 
 
@@ -84,6 +85,7 @@ def _hp(**kw):
     ({"master": 0}, {}, "non-NULL"),
     ({"exp_avg": 8194}, {}, "aligned"),
     ({"max_grads": 65}, {}, "max_grads"),
+    ({"flags": 2}, {}, "flags"),
     ({"wd": float("inf")}, {}, "weight decay"),
 ])
 def test_create_rejects_invalid_arguments_before_cuda(desc_kw, hp_kw, why):
@@ -118,6 +120,12 @@ def test_null_handle_calls():
     assert L.neox_shard_get_state(None, None, None, None) == _abi.NEOX_ERR_INVALID_ARGUMENT
     assert L.neox_shard_set_hparams(None, None) == _abi.NEOX_ERR_INVALID_ARGUMENT
     assert L.neox_shard_scratch_bytes(None) == 0
+    assert L.neox_shard_get_hysteresis(None, None) == _abi.NEOX_ERR_INVALID_ARGUMENT
+    assert L.neox_shard_set_hysteresis(None, 1) == _abi.NEOX_ERR_INVALID_ARGUMENT
+    assert L.neox_ipc_export(None, None, None) == _abi.NEOX_ERR_INVALID_ARGUMENT
+    assert L.neox_ipc_open(None, None) == _abi.NEOX_ERR_INVALID_ARGUMENT
+    assert L.neox_ipc_close(None) == _abi.NEOX_ERR_INVALID_ARGUMENT
+    assert "non-NULL" in _abi.lib().neox_ipc_last_error().decode()
     L.neox_shard_destroy(None)
 
 

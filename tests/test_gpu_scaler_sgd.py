@@ -58,6 +58,20 @@ def test_sgd_bit_exact_clip_off(wbf16, gbf16, K, max_grads, offsets):
     c.close()
 
 
+@pytest.mark.parametrize("wbf16,offset", [(False, 0), (True, 5)])
+def test_sgd_unrolled_loop_bit_exact(wbf16, offset):
+    """A shard long enough that every thread runs the SGD kernel's four-stride
+    batches (more than 4 x resident threads x 8 elements), plus the one-stride
+    remainder, the peeled head and the ragged tail."""
+    torch.cuda.set_device(0)
+    n = 6_000_007
+    c = ShardCase(n, wbf16=wbf16, gbf16=wbf16, offsets={"all": offset}, seed=46, lr=2e-2,
+                  hp=Hparams(clip_norm=0.0, init_scale=2.0 ** 12, optimizer="sgd"),
+                  segments=[(0, 1_000_000, 0.1), (1_000_000, 3, 0.0), (1_000_003, n - 1_000_003, 0.1)])
+    _run(c, 3, overflows={2}, exact=True)
+    c.close()
+
+
 def test_sgd_with_clip_overflow_and_hysteresis():
     torch.cuda.set_device(0)
     # Large gradients (norm about 500, so the clip is active) at a scale that
@@ -176,3 +190,43 @@ def test_multi_hysteresis_bit_exact():
     c.shard.set_state(2.0 ** 10, 0, info.t)
     assert c.shard.get_hysteresis() == 3
     c.shard.close()
+
+
+def test_checkpoint_resume_keeps_the_hysteresis_count():
+    """N steps, state_dict() + the state arrays, destroy, re-create,
+    load_state_dict(), M more steps == N + M uninterrupted steps, byte for
+    byte.  The count is mid-way at the split (two overflows of three
+    tolerated), so a resume that refilled it would back off one step later."""
+    n = 200_003
+    hp = Hparams(init_scale=2.0 ** 12, scale_window=4, hysteresis=3)
+    overflows = {2, 3, 5}
+
+    def run(split, exact_count=True):
+        c = ShardCase(n, hp=hp, lr=6e-4, seed=47)
+        for s in range(1, 9):
+            if s == split:
+                saved = [x.t.clone() for x in (c.master, c.m, c.v, c.w)]
+                sd = c.shard.state_dict()
+                assert sd["hysteresis_count"] == 1
+                c.shard.close()
+                for x, y in zip((c.master, c.m, c.v, c.w), saved):
+                    x.t.copy_(y)
+                c.shard = NeoxShard(c.master.t, c.m.t, c.v.t, hp, weight_decay=0.1)
+                if exact_count:
+                    c.shard.load_state_dict(sd)
+                else:   # a scaler reset instead: the count is refilled
+                    c.shard.set_state(sd["loss_scale"], sd["good_steps"], sd["applied_steps"])
+            c.gen_normal(s, 1e-3)
+            if s in overflows:
+                c.inject(s)
+            c.step()
+        out = [x.t.clone() for x in (c.master, c.m, c.v, c.w)], c.shard.state_dict()
+        c.close()
+        return out
+
+    (a, sa), (b, sb) = run(None), run(4)
+    assert sa == sb
+    for x, y in zip(a, b):
+        assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))
+    _, sr = run(4, exact_count=False)
+    assert sr["loss_scale"] == 2 * sa["loss_scale"]   # the refilled count tolerated step 5's overflow
