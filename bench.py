@@ -311,11 +311,11 @@ def build_gpu_workload(wl, rank, optimizer="adamw"):
     scale = wl.bench_scale or wl.init_scale
     master = _at_offset(n, torch.float32, off)
     synth.gpu_master_normal(master, wl.master_sigma, seed)
-    for off, cnt, _, init in (wl.segments or []):
+    for s_off, cnt, _, init in (wl.segments or []):
         if init == "zero":
-            master[off:off + cnt].zero_()
+            master[s_off:s_off + cnt].zero_()
         elif init == "one":
-            master[off:off + cnt].fill_(1.0)
+            master[s_off:s_off + cnt].fill_(1.0)
     m = _at_offset(n, torch.float32, off).zero_()
     v = _at_offset(n, torch.float32, off).zero_()
     params = _at_offset(n, dt, off)

@@ -153,11 +153,13 @@ neox_status neox_shard_create(const neox_shard_desc* desc, const neox_hparams* h
  *   lr:        learning rate of this step, finite and >= 0;
  *   out:       host result, filled on NEOX_OK.
  * Arrays may start at any element offset: when every array has the same
- * element offset from a 128-byte line the kernels peel a head of up to 63
- * elements and stream whole lines with 16-byte vectors; with only a common
- * 16-byte residue they peel less; otherwise they fall back to narrower
- * vectors.  The results are the same in every case.  The call is stream-ordered and returns after the step
- * has finished on the GPU (it synchronises cuda_stream only).  Overflow is
+ * element offset from a 1024-byte boundary the kernels peel a head of up to
+ * 511 elements and stream from that common boundary with 16-byte vectors
+ * (or the coarsest common 512-, 256- or 128-byte boundary); with only a
+ * common 16-byte residue they peel less; otherwise they fall back to
+ * narrower vectors.  The results are the same in every case.  The call is
+ * stream-ordered and returns after the step has finished on the GPU (it
+ * synchronises cuda_stream only).  Overflow is
  * not an error: it returns NEOX_OK with out->overflow = 1.  On
  * NEOX_ERR_INVALID_ARGUMENT nothing was launched; on NEOX_ERR_CUDA the shard
  * state is undefined. */

@@ -311,6 +311,8 @@ sgd_kernel(GradPtrs gp, int K, const float* __restrict__ acc, Layout L, AdamArgs
 
 // ====================================================================== host
 
+constexpr unsigned long long kAccPad = 256;  // floats of slack: the buffer is shifted by up to 1 KB
+
 struct neox_shard {
     int device = 0;
     int sm_count = 0;
@@ -334,7 +336,7 @@ struct neox_shard {
     unsigned long long* d_seg_end = nullptr;
     float* d_seg_wd = nullptr;
     int nsegs = 0;
-    float* d_acc = nullptr;  // FP32 sum of K >= 5 buffers (numel + 32 floats)
+    float* d_acc = nullptr;  // FP32 sum of the K buffers (numel + kAccPad floats)
     DevScalars* h_sc = nullptr;  // pinned result slot
     unsigned long long owned_bytes = 0;
     // profiling
@@ -499,9 +501,9 @@ neox_status enqueue_step(neox_shard* h, const void* const* grads, int32_t num_gr
     Layout L = h->numel > 0 ? choose_layout(h->numel, a16, num_grads + 1 + h->wcopies.n, a32, 3, vec)
                             : Layout{0, 0, 0, 0};
     float* acc = nullptr;
-    if (use_acc) {
-        const unsigned long long hh = L.head % 32;
-        acc = h->d_acc + ((32 - hh) % 32);  // &acc[head] sits on a 128-byte line
+    if (use_acc) {  // shift the buffer so that &acc[head] sits on a 1024-byte boundary, like the other arrays
+        const uintptr_t a = (uintptr_t)(h->d_acc + L.head);
+        acc = h->d_acc + ((1024u - a % 1024u) % 1024u) / sizeof(float);
     }
 
     ScalerArgs sa;
@@ -683,8 +685,8 @@ neox_status neox_shard_create(const neox_shard_desc* d, const neox_hparams* hp, 
         if ((e = cudaMalloc(&h->d_seg_wd, sizeof(float) * nsegs)) != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMalloc segments"); goto done; }
         bytes += (sizeof(unsigned long long) + sizeof(float)) * nsegs;
         if ((h->max_grads >= 5 || h->accumulate) && h->numel > 0) {
-            if ((e = cudaMalloc(&h->d_acc, sizeof(float) * (h->numel + 32))) != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMalloc accumulation buffer"); goto done; }
-            bytes += sizeof(float) * (h->numel + 32);
+            if ((e = cudaMalloc(&h->d_acc, sizeof(float) * (h->numel + kAccPad))) != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMalloc accumulation buffer"); goto done; }
+            bytes += sizeof(float) * (h->numel + kAccPad);
         }
         h->owned_bytes = bytes;
         if ((e = cudaMallocHost(&h->h_sc, sizeof(DevScalars))) != cudaSuccess) { st = cuda_fail(nullptr, e, "cudaMallocHost"); goto done; }
