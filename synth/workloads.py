@@ -121,5 +121,13 @@ def pythia_2layer() -> Workload:
     return pythia_1p4b(layers=2)
 
 
+def accum8_small() -> Workload:
+    """The 8-buffer recipe at 2^26 parameters (2.4 GB on the device with the
+    FP32 sum buffer): a size that detailed profiler captures handle."""
+    import dataclasses
+    return dataclasses.replace(accum8_predivide(numel=1 << 26), name="accum8_t3_predivide8_fp16_2e26")
+
+
 ALL = {"tiny": tiny, "pythia_1p4b": pythia_1p4b, "neox20b_slice": neox20b_zero1_slice,
-       "accum8": accum8_predivide, "opt_5b": opt_style_5b, "pythia_2layer": pythia_2layer}
+       "accum8": accum8_predivide, "opt_5b": opt_style_5b, "pythia_2layer": pythia_2layer,
+       "accum8_small": accum8_small}
