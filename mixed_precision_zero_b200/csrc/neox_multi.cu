@@ -41,14 +41,29 @@ struct alignas(16) MtTensor {
     float* m;
     float* v;
     uint16_t* w;
-    unsigned long long numel, head, nvec, tail0;
+    unsigned long long numel, head, nvec;  // the vectors are [head, head + nvec * vec)
     float wd;
     int vec;
     int gbase;  // the tensor's K gradient pointers are gtab[gbase .. gbase + K)
     int pad_;
+    // The vectors of all earlier tensors.  A pass's grid-stride starts this
+    // tensor where the previous one left off (this count modulo the pass's
+    // thread count), so the tensors' vectors are dealt to the threads as one
+    // sequence: no thread takes the remainder of every tensor.
+    unsigned long long before;
 };
 
 static_assert(sizeof(MtTensor) % 16 == 0, "descriptors are copied as 16-byte words");
+
+// This thread's first vector of a tensor that follows `before` vectors of
+// earlier tensors (THREADS x gridDim.x threads in all).
+template <int THREADS>
+__device__ __forceinline__ unsigned long long rotated_start(unsigned long long before) {
+    const unsigned long long n = (unsigned long long)gridDim.x * THREADS;
+    const unsigned long long g = (unsigned long long)blockIdx.x * THREADS + threadIdx.x;
+    const unsigned long long r = before % n;
+    return g >= r ? g - r : g + n - r;
+}
 
 // Copy descriptors [base, base + cnt) into shared memory (all threads).  A
 // warp then reads each tensor's pointers from shared memory instead of
@@ -70,7 +85,7 @@ __device__ __forceinline__ void mt_p1_tensor(const GradTab& gp, int K_rt, const 
     const int K = KFIX ? KFIX : K_rt;
     constexpr int U = KFIX ? 4 : 2;
     const unsigned long long stride = (unsigned long long)gridDim.x * kMtThreads1;
-    unsigned long long v = (unsigned long long)blockIdx.x * kMtThreads1 + threadIdx.x;
+    unsigned long long v = rotated_start<kMtThreads1>(T.before);
     for (; v + (U - 1) * stride < T.nvec; v += U * stride) {
         float g[U][VEC];
         ingest_batch<G, VEC, U>(gp, K, T.head + v * VEC, stride * VEC, inv_pre, inv_us, g);
@@ -124,9 +139,10 @@ mt_stats_kernel(const MtTensor* __restrict__ tens, int ntensors, const uint16_t*
         if (K == 1) mt_p1_dispatch<G, 1>(T, gp, K, sa.inv_pre, inv_us, s, bad);
         else mt_p1_dispatch<G, 0>(T, gp, K, sa.inv_pre, inv_us, s, bad);
         if ((unsigned)ti % gridDim.x == blockIdx.x) {  // this tensor's head and tail
-            const unsigned long long extra = T.head + (T.numel - T.tail0);
+            const unsigned long long tail0 = T.head + T.nvec * T.vec;
+            const unsigned long long extra = T.head + (T.numel - tail0);
             for (unsigned long long j = threadIdx.x; j < extra; j += kMtThreads1) {
-                const unsigned long long i = j < T.head ? j : T.tail0 + (j - T.head);
+                const unsigned long long i = j < T.head ? j : tail0 + (j - T.head);
                 float g[1];
                 ingest<G, 1>(gp, K, i, sa.inv_pre, inv_us, g);
                 s += vec_sumsq<1>(g, bad);
@@ -151,7 +167,26 @@ __device__ __forceinline__ void mt_p2_tensor(const GradTab& gp, int K_rt, const 
     float* __restrict__ v = T.v;
     uint16_t* __restrict__ w = T.w;
     const unsigned long long nvec = T.nvec, head = T.head;
-    for (unsigned long long vi = (unsigned long long)blockIdx.x * kMtThreads3 + threadIdx.x; vi < nvec; vi += stride) {
+    unsigned long long vi = rotated_start<kMtThreads3>(T.before);
+    if constexpr (SGD) {
+        // kUnrollSgd strides in flight per thread, as in the flat SGD pass
+        // (its loads are too few to cover the memory latency one at a time).
+        constexpr int U = kUnrollSgd;
+        for (; vi + (U - 1) * stride < nvec; vi += U * stride) {
+            float g[U][VEC], p[U][VEC];
+            ingest_batch<G, VEC, U>(gp, K, head + vi * VEC, stride * VEC, a.inv_pre, inv_us, g);
+#pragma unroll
+            for (int u = 0; u < U; u++) ld32<VEC>(master + head + (vi + u * stride) * VEC, p[u]);
+#pragma unroll
+            for (int u = 0; u < U; u++) {
+                const unsigned long long i = head + (vi + u * stride) * VEC;
+                sgd_vec<VEC>(g[u], keep, c, a.lr, p[u]);
+                st32<VEC>(master + i, p[u]);
+                st16<W, VEC>(w + i, p[u]);
+            }
+        }
+    }
+    for (; vi < nvec; vi += stride) {
         const unsigned long long i = head + vi * VEC;
         float g[VEC], p[VEC], mm[VEC], vv[VEC];
         ingest<G, VEC>(gp, K, i, a.inv_pre, inv_us, g);
@@ -212,9 +247,10 @@ __device__ __forceinline__ void mt_update(const MtTensor* __restrict__ tens, int
         if (K == 1) mt_p2_dispatch<SGD, G, W, 1>(T, gp, K, keep1, c, inv_us, a);
         else mt_p2_dispatch<SGD, G, W, 0>(T, gp, K, keep1, c, inv_us, a);
         if ((unsigned)ti % gridDim.x == blockIdx.x) {  // this tensor's head and tail
-            const unsigned long long extra = T.head + (T.numel - T.tail0);
+            const unsigned long long tail0 = T.head + T.nvec * T.vec;
+            const unsigned long long extra = T.head + (T.numel - tail0);
             for (unsigned long long j = threadIdx.x; j < extra; j += kMtThreads3) {
-                const unsigned long long i = j < T.head ? j : T.tail0 + (j - T.head);
+                const unsigned long long i = j < T.head ? j : tail0 + (j - T.head);
                 float g[1], p[1] = {T.master[i]}, keep[1] = {keep1};
                 ingest<G, 1>(gp, K, i, a.inv_pre, inv_us, g);
                 if constexpr (SGD) {
@@ -269,8 +305,9 @@ struct neox_multi {
     neox_dtype wdtype = NEOX_FP16, gdtype = NEOX_FP16;
     neox_hparams hp{};
     unsigned long long numel = 0;
-    unsigned long long max_vecs = 0;  // vectors of the largest tensor
-    int grid2 = 1;                    // pass-2 grid (resident blocks, set at create)
+    unsigned long long total_vecs = 0;  // vectors of all tensors
+    int grid1 = 1;                      // pass-1 grid (set at create)
+    int grid2 = 1, grid2_sgd = 1;       // pass-2 grids of the two update rules (set at create)
     float scale = 1.0f;
     int32_t good = 0;
     long long t = 0;
@@ -345,18 +382,17 @@ std::string build_tables(const neox_tensor_set* set, std::vector<MtTensor>& tens
         T.w = static_cast<uint16_t*>(d.params);
         T.head = L.head;
         T.nvec = L.nvec;
-        T.tail0 = L.tail0;
         T.vec = vec;
     }
     return "";
 }
 
-// Resident-grid size for the multi-tensor kernels (at most enough blocks to
-// cover the largest tensor once).
+// Resident-grid size for the multi-tensor kernels (at most one vector of all
+// the tensors' vectors per thread).
 template <class Kern>
-int mt_grid(Kern kernel, int threads, unsigned long long max_vecs, int sm_count, int cap) {
+int mt_grid(Kern kernel, int threads, unsigned long long total_vecs, int sm_count, int cap) {
     unsigned long long g = (unsigned long long)sm_count * occupancy(kernel, threads);
-    const unsigned long long want = (max_vecs + threads - 1) / threads;
+    const unsigned long long want = (total_vecs + threads - 1) / threads;
     if (g > want) g = want;
     if (g > (unsigned long long)cap) g = cap;
     return g < 1 ? 1 : (int)g;
@@ -376,14 +412,14 @@ neox_status mt_enqueue(neox_multi* h, float lr, const float* lr_dev, cudaStream_
     cudaError_t e;
     {
         auto k1 = h->gdtype == NEOX_FP16 ? mt_stats_kernel<F16> : mt_stats_kernel<BF16>;
-        const int grid = mt_grid(k1, kMtThreads1, h->max_vecs, h->sm_count, h->max_parts);
+        const int grid = h->grid1;
         k1<<<grid, kMtThreads1, 0, st>>>(h->d_tens, h->ntensors, h->d_gtab, h->K, sa, h->d_part_s, h->d_part_b,
                                          h->d_sc);
         if ((e = cudaGetLastError()) != cudaSuccess) return mcuda_fail(h, e, "pass-1 launch");
     }
     if (h->numel > 0) {
         const MtUpdateKernel k2 = mt_update_kernel(h->hp.optimizer == NEOX_SGD, h->gdtype, h->wdtype);
-        const int grid = h->grid2;
+        const int grid = h->hp.optimizer == NEOX_SGD ? h->grid2_sgd : h->grid2;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(grid);
         cfg.blockDim = dim3(kMtThreads3);
@@ -448,9 +484,8 @@ neox_status neox_multi_create(const neox_tensor_set* set, const neox_hparams* hp
     h->scale = hp->init_scale;
     for (const auto& T : tens) {
         h->numel += T.numel;
-        if (T.nvec > h->max_vecs) h->max_vecs = T.nvec;
+        h->total_vecs += T.nvec;
     }
-    h->tens = tens;
     neox_status st = NEOX_OK;
     cudaError_t e;
     {
@@ -477,13 +512,6 @@ neox_status neox_multi_create(const neox_tensor_set* set, const neox_hparams* hp
             st = mcuda_fail(nullptr, e, "allocation");
             goto done;
         }
-        if ((!tens.empty() && (e = cudaMemcpy(h->d_tens, tens.data(), sizeof(MtTensor) * tens.size(),
-                                              cudaMemcpyHostToDevice)) != cudaSuccess) ||
-            (!gtab.empty() && (e = cudaMemcpy(h->d_gtab, gtab.data(), sizeof(void*) * gtab.size(),
-                                              cudaMemcpyHostToDevice)) != cudaSuccess)) {
-            st = mcuda_fail(nullptr, e, "copying the tensor tables");
-            goto done;
-        }
         DevScalars init{};
         init.scale = hp->init_scale;
         init.scale_used = hp->init_scale;
@@ -497,17 +525,36 @@ neox_status neox_multi_create(const neox_tensor_set* set, const neox_hparams* hp
         const MtUpdateKernel k2 = mt_update_kernel(false, h->gdtype, h->wdtype);
         const MtUpdateKernel k2s = mt_update_kernel(true, h->gdtype, h->wdtype);
         const int dyn = (int)(sizeof(MtTensor) * kMtDescBatch3);
-        int occ = 0;
+        int occ = 0, occ_sgd = 0;
         if ((e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn)) != cudaSuccess ||
             (e = cudaFuncSetAttribute(k2s, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn)) != cudaSuccess ||
-            (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k2, kMtThreads3, dyn)) != cudaSuccess) {
+            (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k2, kMtThreads3, dyn)) != cudaSuccess ||
+            (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_sgd, k2s, kMtThreads3, dyn)) != cudaSuccess) {
             st = mcuda_fail(nullptr, e, "configuring the update kernel");
             goto done;
         }
+        const unsigned long long want2 = (h->total_vecs + kMtThreads3 - 1) / kMtThreads3;
         unsigned long long g2 = (unsigned long long)h->sm_count * (occ < 1 ? 1 : occ);
-        const unsigned long long want2 = (h->max_vecs + kMtThreads3 - 1) / kMtThreads3;
+        unsigned long long g2s = (unsigned long long)h->sm_count * (occ_sgd < 1 ? 1 : occ_sgd);
         if (g2 > want2) g2 = want2;
+        if (g2s > want2) g2s = want2;
         h->grid2 = g2 < 1 ? 1 : (int)g2;
+        h->grid2_sgd = g2s < 1 ? 1 : (int)g2s;
+        auto k1 = h->gdtype == NEOX_FP16 ? mt_stats_kernel<F16> : mt_stats_kernel<BF16>;
+        h->grid1 = mt_grid(k1, kMtThreads1, h->total_vecs, h->sm_count, h->max_parts);
+        unsigned long long before = 0;
+        for (auto& T : tens) {
+            T.before = before;
+            before += T.nvec;
+        }
+        h->tens = tens;
+        if ((!tens.empty() && (e = cudaMemcpy(h->d_tens, tens.data(), sizeof(MtTensor) * tens.size(),
+                                              cudaMemcpyHostToDevice)) != cudaSuccess) ||
+            (!gtab.empty() && (e = cudaMemcpy(h->d_gtab, gtab.data(), sizeof(void*) * gtab.size(),
+                                              cudaMemcpyHostToDevice)) != cudaSuccess)) {
+            st = mcuda_fail(nullptr, e, "copying the tensor tables");
+            goto done;
+        }
     }
 done:
     if (st != NEOX_OK) {

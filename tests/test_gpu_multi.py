@@ -191,3 +191,40 @@ def test_multi_rejects_bad_tensors():
     with pytest.raises(NeoxError) as ei:
         _abi.neox_multi_create(ts, Hparams().c(), 0)
     assert ei.value.status == _abi.NEOX_ERR_INVALID_ARGUMENT
+
+
+@pytest.mark.parametrize("optimizer", ["adamw", "sgd"])
+def test_multi_large_tensors_match_flat(optimizer):
+    """Tensors many grid strides long (the SGD form's four-stride batches, the
+    rotated starts wrapping around the thread count) against the flat step on
+    the same bytes, which is itself checked against the oracle: with clipping
+    off the two give identical state."""
+    torch.cuda.set_device(0)
+    sizes = [3_000_017, 5, 2_000_003, 1_048_576, 777]
+    wds = [0.1, 0.0, 0.1, 0.05, 0.0]
+    segs, off = [], 0
+    for n_, wd in zip(sizes, wds):
+        segs.append((off, n_, wd))
+        off += n_
+    n = off
+    hp = Hparams(clip_norm=0.0, init_scale=2.0 ** 10, optimizer=optimizer)
+    master = torch.empty(n, dtype=torch.float32, device="cuda")
+    synth.gpu_master_normal(master, 0.02, 12)
+    a = [master, torch.zeros_like(master), torch.zeros_like(master), master.to(torch.float16)]
+    b = [x.clone() for x in a]
+    gs = [torch.empty(n, dtype=torch.float16, device="cuda") for _ in range(2)]
+    flat = NeoxShard(a[0], a[1], a[2], hp, segments=segs, max_grads=2)
+    multi = NeoxMultiShard([{"master": b[0][o:o + k], "exp_avg": b[1][o:o + k], "exp_avg_sq": b[2][o:o + k],
+                             "params": b[3][o:o + k], "grads": [g[o:o + k] for g in gs], "weight_decay": w}
+                            for o, k, w in segs], hp)
+    for s in range(1, 5):
+        for k, g in enumerate(gs):
+            synth.gpu_grad_normal16(g, 2e-3, 2.0 ** 10, 12, k, s)
+        ra = flat.step(gs, a[3], 1e-2)
+        rb = multi.step(1e-2)
+        assert ra.overflow == rb.overflow == 0 and ra.applied_steps == rb.applied_steps
+        assert abs(ra.grad_norm - rb.grad_norm) <= 1e-6 * ra.grad_norm
+    for x, y in zip(a, b):
+        assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))
+    flat.close()
+    multi.close()
