@@ -12,6 +12,8 @@
 
 #include <cmath>
 #include <cstdint>
+#include <mutex>
+#include <unordered_map>
 
 namespace {
 
@@ -19,7 +21,7 @@ constexpr int kMaxGrads = 64;
 constexpr int kThreads1 = 512;   // pass-1 block
 constexpr int kUnroll1 = 4;      // pass-1 vectors in flight per thread
 constexpr int kThreads3 = 256;   // pass-2 block
-constexpr int kUnroll3 = 1;      // pass-2 vectors in flight per thread (AdamW)
+constexpr int kChunk3 = 4;       // pass-2 (AdamW) vectors per thread in each dynamically taken chunk
 constexpr int kUnrollSgd = 4;    // pass-2 vectors in flight per thread (SGD): measured 6.25 TB/s against 5.83 at 1
 constexpr int kMaxBlocksPerSm = 32;
 
@@ -51,7 +53,7 @@ struct __align__(64) DevScalars {
     float bc2_sqrt;        // device-computed fl32(sqrt(bc2)) of the last step (asynchronous steps)
     float lr;              // learning rate of the last step (asynchronous steps)
     int32_t hyst;          // overflows still tolerated before the next back-off
-    int32_t pad_;
+    unsigned int chunk_next;   // pass-2 work counter: zeroed before every pass 2
 };
 static_assert(sizeof(DevScalars) == 64, "DevScalars is one 64-byte block");
 
@@ -442,6 +444,7 @@ __device__ __forceinline__ void finish_pass1(double s, int bad, double* __restri
         decide_step(sc, sa, s, bad);
     }
     sc->blocks_done = 0;
+    sc->chunk_next = 0;  // for the pass 2 that follows (it waits for this grid to finish)
 }
 
 template <int VEC>
@@ -477,7 +480,10 @@ __device__ __forceinline__ void sgd_vec(const float (&g)[VEC], const float (&kee
 // The decision of a split step from all-reduced statistics {sum of squares,
 // number of ranks that saw a non-finite value}.  One thread.
 __global__ void decide_kernel(DevScalars* __restrict__ sc, ScalerArgs sa, const double* __restrict__ stats) {
-    if (threadIdx.x == 0 && blockIdx.x == 0) decide_step(sc, sa, stats[0], stats[1] != 0.0);
+    if (threadIdx.x == 0 && blockIdx.x == 0) {
+        decide_step(sc, sa, stats[0], stats[1] != 0.0);
+        sc->chunk_next = 0;
+    }
 }
 
 // ---------------------------------------------------------------- host helpers
@@ -596,15 +602,21 @@ Layout choose_layout(unsigned long long n, const uintptr_t* a16, int n16, const 
     return make(1, 0);  // unreachable: VEC = 1 always fits
 }
 
+// Resident blocks per SM of `kernel` at `threads` per block (no dynamic
+// shared memory), cached per kernel: kernels of one signature share a
+// function-pointer type, so the cache is keyed by the kernel's address.
 template <class K>
 int occupancy(K kernel, int threads) {
-    static int cached = 0;
-    if (cached == 0) {
-        int occ = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, threads, 0) != cudaSuccess || occ < 1) occ = 1;
-        cached = occ;
-    }
-    return cached;
+    static std::mutex mu;
+    static std::unordered_map<const void*, int> cache;
+    const void* key = reinterpret_cast<const void*>(kernel);
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, threads, 0) != cudaSuccess || occ < 1) occ = 1;
+    cache.emplace(key, occ);
+    return occ;
 }
 
 template <class K>

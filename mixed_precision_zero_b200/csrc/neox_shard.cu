@@ -134,28 +134,51 @@ __device__ __forceinline__ void store_copies(const WeightCopies& wc, unsigned lo
         if (d < wc.n) st16<W, VEC>(wc.p[d] + i, p);
 }
 
-// The vector loop of pass 2 (KFIX as in pass1_vectors).  SGD: plain SGD,
-// which neither reads nor writes m and v; else AdamW.
-template <bool SGD, class G, class W, int VEC, bool READ_ACC, int KFIX, bool COPIES>
+// The decay factor fl32(1 - fl32(lr * wd)) of each of the VEC elements at i
+// (a vector may straddle a segment boundary).  The cursor only moves forward.
+template <int VEC>
+__device__ __forceinline__ void keep_at(SegCursor& cur, unsigned long long i, const unsigned long long* seg_end,
+                                        const float* seg_wd, int nsegs, float lr, float (&keep)[VEC]) {
+    if (i >= cur.end) seg_seek(cur, i, seg_end, seg_wd, nsegs, lr);
+    if (i + VEC <= cur.end) {
+#pragma unroll
+        for (int e = 0; e < VEC; e++) keep[e] = cur.keep;
+    } else {
+#pragma unroll
+        for (int e = 0; e < VEC; e++) {
+            if (i + e >= cur.end) seg_seek(cur, i + e, seg_end, seg_wd, nsegs, lr);
+            keep[e] = cur.keep;
+        }
+    }
+}
+
+// The vector loop of pass 2 (KFIX as in pass1_vectors).
+//  AdamW: blocks take chunks of kChunk3 x kThreads3 vectors from a counter in
+//    the scalar block (zeroed by pass 1's last block, which this grid waits
+//    for).  Blocks whose memory traffic is served faster take more chunks;
+//    with the static grid-stride the pass that reads the FP32 sum left its
+//    SMs unevenly busy and ran at 5.6 TB/s, against 6.8 with chunks.
+//    CHUNKED = false (shards of less than one chunk per block, chosen on the
+//    host) keeps the one-vector grid-stride: there a chunk's kChunk3
+//    dependent iterations would be the whole latency.
+//  SGD: the static grid-stride, kUnrollSgd strides in flight per thread (its
+//    loads are too few per vector to cover the memory latency one at a time).
+template <bool SGD, class G, class W, int VEC, bool READ_ACC, int KFIX, bool COPIES, bool CHUNKED>
 __device__ __forceinline__ void pass2_vectors(const GradPtrs& gp, int K_rt, const float* __restrict__ acc,
                                               const Layout& L, const AdamArgs& a, float c, float inv_us,
                                               float* __restrict__ master, float* __restrict__ m,
                                               float* __restrict__ v, uint16_t* __restrict__ w,
                                               const unsigned long long* __restrict__ seg_end,
-                                              const float* __restrict__ seg_wd, int nsegs, const WeightCopies& wc) {
+                                              const float* __restrict__ seg_wd, int nsegs, const WeightCopies& wc,
+                                              DevScalars* __restrict__ sc) {
     const int K = KFIX ? KFIX : K_rt;
-    constexpr int U = SGD ? kUnrollSgd : kUnroll3;
-    const unsigned long long stride = (unsigned long long)gridDim.x * kThreads3;
-    unsigned long long v0 = (unsigned long long)blockIdx.x * kThreads3 + threadIdx.x;
     SegCursor cur{0, 0ull, 1.0f};
-    if (v0 < L.nvec) seg_seek(cur, L.head + v0 * VEC, seg_end, seg_wd, nsegs, a.lr);
-
-    unsigned long long vi = v0;
-    // U strides per iteration: every load of the batch is issued before
-    // the first update, to keep more bytes in flight per thread.
-    if constexpr (U > 1) {
+    if constexpr (SGD) {
+        constexpr int U = kUnrollSgd;
+        const unsigned long long stride = (unsigned long long)gridDim.x * kThreads3;
+        unsigned long long vi = (unsigned long long)blockIdx.x * kThreads3 + threadIdx.x;
         for (; vi + (U - 1) * stride < L.nvec; vi += U * stride) {
-            float g[U][VEC], p[U][VEC], mm[U][VEC], vv[U][VEC];
+            float g[U][VEC], p[U][VEC];
             if constexpr (READ_ACC) {
 #pragma unroll
                 for (int u = 0; u < U; u++) ld32<VEC>(acc + L.head + (vi + u * stride) * VEC, g[u]);
@@ -163,87 +186,90 @@ __device__ __forceinline__ void pass2_vectors(const GradPtrs& gp, int K_rt, cons
                 ingest_batch<G, VEC, U>(gp, K, L.head + vi * VEC, stride * VEC, a.inv_pre, inv_us, g);
             }
 #pragma unroll
-            for (int u = 0; u < U; u++) {
-                const unsigned long long i = L.head + (vi + u * stride) * VEC;
-                ld32<VEC>(master + i, p[u]);
-                if constexpr (!SGD) {
-                    ld32<VEC>(m + i, mm[u]);
-                    ld32<VEC>(v + i, vv[u]);
-                }
-            }
+            for (int u = 0; u < U; u++) ld32<VEC>(master + L.head + (vi + u * stride) * VEC, p[u]);
 #pragma unroll
             for (int u = 0; u < U; u++) {
                 const unsigned long long i = L.head + (vi + u * stride) * VEC;
                 float keep[VEC];
-                if (i >= cur.end) seg_seek(cur, i, seg_end, seg_wd, nsegs, a.lr);
-                if (i + VEC <= cur.end) {
-#pragma unroll
-                    for (int e = 0; e < VEC; e++) keep[e] = cur.keep;
-                } else {
-#pragma unroll
-                    for (int e = 0; e < VEC; e++) {
-                        if (i + e >= cur.end) seg_seek(cur, i + e, seg_end, seg_wd, nsegs, a.lr);
-                        keep[e] = cur.keep;
-                    }
-                }
-                if constexpr (SGD) {
-                    sgd_vec<VEC>(g[u], keep, c, a.lr, p[u]);
-                    st32<VEC>(master + i, p[u]);
-                } else {
-                    adam_vec<VEC>(g[u], keep, c, a, p[u], mm[u], vv[u]);
-                    st32<VEC>(master + i, p[u]);
-                    st32<VEC>(m + i, mm[u]);
-                    st32<VEC>(v + i, vv[u]);
-                }
+                keep_at<VEC>(cur, i, seg_end, seg_wd, nsegs, a.lr, keep);
+                sgd_vec<VEC>(g[u], keep, c, a.lr, p[u]);
+                st32<VEC>(master + i, p[u]);
                 st16<W, VEC>(w + i, p[u]);
                 if constexpr (COPIES) store_copies<W, VEC>(wc, i, p[u]);
             }
         }
-    }
-    for (; vi < L.nvec; vi += stride) {
-        const unsigned long long i = L.head + vi * VEC;
-        float g[VEC], p[VEC], mm[VEC], vv[VEC], keep[VEC];
-        if constexpr (READ_ACC) ld32<VEC>(acc + i, g);
-        else ingest<G, VEC>(gp, K, i, a.inv_pre, inv_us, g);
-        ld32<VEC>(master + i, p);
-        if constexpr (!SGD) {
-            ld32<VEC>(m + i, mm);
-            ld32<VEC>(v + i, vv);
-        }
-        if (i >= cur.end) seg_seek(cur, i, seg_end, seg_wd, nsegs, a.lr);
-        if (i + VEC <= cur.end) {
-#pragma unroll
-            for (int e = 0; e < VEC; e++) keep[e] = cur.keep;
-        } else {
-#pragma unroll
-            for (int e = 0; e < VEC; e++) {
-                if (i + e >= cur.end) seg_seek(cur, i + e, seg_end, seg_wd, nsegs, a.lr);
-                keep[e] = cur.keep;
-            }
-        }
-        if constexpr (SGD) {
+        for (; vi < L.nvec; vi += stride) {
+            const unsigned long long i = L.head + vi * VEC;
+            float g[VEC], p[VEC], keep[VEC];
+            if constexpr (READ_ACC) ld32<VEC>(acc + i, g);
+            else ingest<G, VEC>(gp, K, i, a.inv_pre, inv_us, g);
+            ld32<VEC>(master + i, p);
+            keep_at<VEC>(cur, i, seg_end, seg_wd, nsegs, a.lr, keep);
             sgd_vec<VEC>(g, keep, c, a.lr, p);
             st32<VEC>(master + i, p);
-        } else {
+            st16<W, VEC>(w + i, p);
+            if constexpr (COPIES) store_copies<W, VEC>(wc, i, p);
+        }
+    } else if constexpr (!CHUNKED) {
+        const unsigned long long stride = (unsigned long long)gridDim.x * kThreads3;
+        for (unsigned long long vi = (unsigned long long)blockIdx.x * kThreads3 + threadIdx.x; vi < L.nvec;
+             vi += stride) {
+            const unsigned long long i = L.head + vi * VEC;
+            float g[VEC], p[VEC], mm[VEC], vv[VEC], keep[VEC];
+            if constexpr (READ_ACC) ld32<VEC>(acc + i, g);
+            else ingest<G, VEC>(gp, K, i, a.inv_pre, inv_us, g);
+            ld32<VEC>(master + i, p);
+            ld32<VEC>(m + i, mm);
+            ld32<VEC>(v + i, vv);
+            keep_at<VEC>(cur, i, seg_end, seg_wd, nsegs, a.lr, keep);
             adam_vec<VEC>(g, keep, c, a, p, mm, vv);
             st32<VEC>(master + i, p);
             st32<VEC>(m + i, mm);
             st32<VEC>(v + i, vv);
+            st16<W, VEC>(w + i, p);
+            if constexpr (COPIES) store_copies<W, VEC>(wc, i, p);
         }
-        st16<W, VEC>(w + i, p);
-        if constexpr (COPIES) store_copies<W, VEC>(wc, i, p);
+    } else {
+        constexpr unsigned long long kChunk = (unsigned long long)kThreads3 * kChunk3;
+        const unsigned long long nchunks = (L.nvec + kChunk - 1) / kChunk;
+        __shared__ unsigned int chunk_sh;
+        for (;;) {
+            if (threadIdx.x == 0) chunk_sh = atomicAdd(&sc->chunk_next, 1u);
+            __syncthreads();
+            const unsigned long long ch = chunk_sh;
+            __syncthreads();                  // chunk_sh is rewritten by the next iteration
+            if (ch >= nchunks) break;         // uniform across the block
+            for (int k = 0; k < kChunk3; k++) {
+                const unsigned long long vi = ch * kChunk + (unsigned long long)k * kThreads3 + threadIdx.x;
+                if (vi >= L.nvec) break;
+                const unsigned long long i = L.head + vi * VEC;
+                float g[VEC], p[VEC], mm[VEC], vv[VEC], keep[VEC];
+                if constexpr (READ_ACC) ld32<VEC>(acc + i, g);
+                else ingest<G, VEC>(gp, K, i, a.inv_pre, inv_us, g);
+                ld32<VEC>(master + i, p);
+                ld32<VEC>(m + i, mm);
+                ld32<VEC>(v + i, vv);
+                keep_at<VEC>(cur, i, seg_end, seg_wd, nsegs, a.lr, keep);
+                adam_vec<VEC>(g, keep, c, a, p, mm, vv);
+                st32<VEC>(master + i, p);
+                st32<VEC>(m + i, mm);
+                st32<VEC>(v + i, vv);
+                st16<W, VEC>(w + i, p);
+                if constexpr (COPIES) store_copies<W, VEC>(wc, i, p);
+            }
+        }
     }
 }
 
 // The whole of pass 2 for one grid: the vector loop, then (block 0) the
 // peeled head and the ragged tail one element per thread.
-template <bool SGD, class G, class W, int VEC, bool READ_ACC, bool COPIES>
+template <bool SGD, class G, class W, int VEC, bool READ_ACC, bool COPIES, bool CHUNKED>
 __device__ __forceinline__ void update_shard(const GradPtrs& gp, int K, const float* __restrict__ acc,
                                              const Layout& L, const AdamArgs& a_arg, float* __restrict__ master,
                                              float* __restrict__ m, float* __restrict__ v, uint16_t* __restrict__ w,
                                              const unsigned long long* __restrict__ seg_end,
                                              const float* __restrict__ seg_wd, int nsegs,
-                                             const DevScalars* __restrict__ sc, const WeightCopies& wc) {
+                                             DevScalars* __restrict__ sc, const WeightCopies& wc) {
     // Programmatic dependent launch: everything below reads what pass 1 wrote.
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (sc->overflow) return;  // skipped step: nothing is written
@@ -257,11 +283,11 @@ __device__ __forceinline__ void update_shard(const GradPtrs& gp, int K, const fl
     }
 
     if (K == 1)
-        pass2_vectors<SGD, G, W, VEC, READ_ACC, 1, COPIES>(gp, K, acc, L, a, c, inv_us, master, m, v, w, seg_end, seg_wd,
-                                                           nsegs, wc);
+        pass2_vectors<SGD, G, W, VEC, READ_ACC, 1, COPIES, CHUNKED>(gp, K, acc, L, a, c, inv_us, master, m, v, w, seg_end, seg_wd,
+                                                           nsegs, wc, sc);
     else
-        pass2_vectors<SGD, G, W, VEC, READ_ACC, 0, COPIES>(gp, K, acc, L, a, c, inv_us, master, m, v, w, seg_end, seg_wd,
-                                                           nsegs, wc);
+        pass2_vectors<SGD, G, W, VEC, READ_ACC, 0, COPIES, CHUNKED>(gp, K, acc, L, a, c, inv_us, master, m, v, w, seg_end, seg_wd,
+                                                           nsegs, wc, sc);
     if (blockIdx.x == 0) {
         const unsigned long long extra = L.head + (L.n - L.tail0);
         for (unsigned long long j = threadIdx.x; j < extra; j += kThreads3) {
@@ -288,13 +314,14 @@ __device__ __forceinline__ void update_shard(const GradPtrs& gp, int K, const fl
 }
 
 // Pass 2 with AdamW.
-template <class G, class W, int VEC, bool READ_ACC, bool COPIES>
+template <class G, class W, int VEC, bool READ_ACC, bool COPIES, bool CHUNKED>
 __global__ void __launch_bounds__(kThreads3)
 adam_kernel(GradPtrs gp, int K, const float* __restrict__ acc, Layout L, AdamArgs a,
             float* __restrict__ master, float* __restrict__ m, float* __restrict__ v, uint16_t* __restrict__ w,
             const unsigned long long* __restrict__ seg_end, const float* __restrict__ seg_wd, int nsegs,
-            const DevScalars* __restrict__ sc, WeightCopies wc) {
-    update_shard<false, G, W, VEC, READ_ACC, COPIES>(gp, K, acc, L, a, master, m, v, w, seg_end, seg_wd, nsegs, sc, wc);
+            DevScalars* __restrict__ sc, WeightCopies wc) {
+    update_shard<false, G, W, VEC, READ_ACC, COPIES, CHUNKED>(gp, K, acc, L, a, master, m, v, w, seg_end, seg_wd, nsegs,
+                                                              sc, wc);
 }
 
 // Pass 2 with plain SGD (m and v are not touched).
@@ -303,8 +330,9 @@ __global__ void __launch_bounds__(kThreads3)
 sgd_kernel(GradPtrs gp, int K, const float* __restrict__ acc, Layout L, AdamArgs a,
            float* __restrict__ master, float* __restrict__ m, float* __restrict__ v, uint16_t* __restrict__ w,
            const unsigned long long* __restrict__ seg_end, const float* __restrict__ seg_wd, int nsegs,
-           const DevScalars* __restrict__ sc, WeightCopies wc) {
-    update_shard<true, G, W, VEC, READ_ACC, COPIES>(gp, K, acc, L, a, master, m, v, w, seg_end, seg_wd, nsegs, sc, wc);
+           DevScalars* __restrict__ sc, WeightCopies wc) {
+    update_shard<true, G, W, VEC, READ_ACC, COPIES, false>(gp, K, acc, L, a, master, m, v, w, seg_end, seg_wd, nsegs,
+                                                           sc, wc);
 }
 
 }  // namespace
@@ -376,8 +404,11 @@ cudaError_t launch_pass2(neox_shard* h, const GradPtrs& gp, int K, const float* 
                          const AdamArgs& a, uint16_t* w, cudaStream_t st) {
     const bool sgd = h->hp.optimizer == NEOX_SGD, copies = h->wcopies.n > 0;
     auto kern = sgd ? (copies ? sgd_kernel<G, W, VEC, ACC, true> : sgd_kernel<G, W, VEC, ACC, false>)
-                    : (copies ? adam_kernel<G, W, VEC, ACC, true> : adam_kernel<G, W, VEC, ACC, false>);
+                    : (copies ? adam_kernel<G, W, VEC, ACC, true, true> : adam_kernel<G, W, VEC, ACC, false, true>);
     const int grid = grid_for(kern, kThreads3, L.nvec, h->sm_count, 1 << 20);
+    // AdamW takes chunks only when the shard has at least one per block
+    if (!sgd && L.nvec < (unsigned long long)grid * kThreads3 * kChunk3)
+        kern = copies ? adam_kernel<G, W, VEC, ACC, true, false> : adam_kernel<G, W, VEC, ACC, false, false>;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kThreads3);
@@ -391,7 +422,7 @@ cudaError_t launch_pass2(neox_shard* h, const GradPtrs& gp, int K, const float* 
     const float* accp = acc;
     const unsigned long long* se = h->d_seg_end;
     const float* sw = h->d_seg_wd;
-    const DevScalars* sc = h->d_sc;
+    DevScalars* sc = h->d_sc;
     return cudaLaunchKernelEx(&cfg, kern, gp, K, accp, L, a, h->master, h->m, h->v, w, se, sw, h->nsegs, sc,
                               h->wcopies);
 }

@@ -358,3 +358,26 @@ def test_weight_copies_receive_the_cast(offsets):
             assert x.guards_intact()
     c.shard.set_weight_copies([])
     c.close()
+
+
+@pytest.mark.parametrize("K,max_grads,offset", [(1, 1, 0), (6, 8, 5), (2, 2, 3)])
+def test_chunked_update_bit_exact(K, max_grads, offset):
+    """A shard of more than one pass-2 chunk per block, so the AdamW pass takes
+    its work from the chunk counter (through the FP32 sum for K = 6): the
+    state equals the oracle byte for byte with clipping off, through an
+    overflowed step, segment boundaries, the peeled head and the ragged tail."""
+    torch.cuda.set_device(0)
+    n = 8_000_011
+    segs = [(0, 1_000_003, 0.1), (1_000_003, 4_097, 0.0), (1_004_100, n - 1_004_100, 0.1)]
+    c = ShardCase(n, K=K, max_grads=max_grads, offsets={"all": offset}, segments=segs, seed=61, lr=1e-3,
+                  hp=Hparams(clip_norm=0.0, predivide=float(K), init_scale=2.0 ** 12, scale_window=2))
+    for s in range(1, 5):
+        c.gen_normal(s, 2e-3)
+        if s == 3:
+            c.inject(s, buffer=K - 1)
+        res, info = c.step()
+        c.check_result(res, info)
+        assert res.overflow == (1 if s == 3 else 0)
+    c.check_state(exact=True)
+    assert c.guards_intact()
+    c.close()
