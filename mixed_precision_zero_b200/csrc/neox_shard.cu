@@ -23,9 +23,12 @@
 //          in a fixed order, so the norm is deterministic, and runs the
 //          loss scaler and the clip coefficient on the device.
 //  pass 2  adam_kernel: one streaming pass over grad (or the FP32 sum),
-//          master, m, v with 16-byte vectors; returns at once when the step
-//          overflowed; AdamW with the clip folded in; writes master, m, v and
-//          the 16-bit working copy with streaming stores.
+//          master, m, v with 16-byte vectors, the blocks taking their work in
+//          chunks from a counter that pass 1 zeroed (so SMs that are served
+//          faster take more); returns at once when the step overflowed; AdamW
+//          with the clip folded in; writes master, m, v and the 16-bit
+//          working copy with streaming stores.  sgd_kernel: the same pass
+//          with plain SGD, which neither reads nor writes m and v.
 // Every FP32 operation of the ingest and of the update uses an explicit
 // round-to-nearest intrinsic (no contraction), in the same order as the plain
 // definition, so for equal clip coefficients the results are bit-exact with
