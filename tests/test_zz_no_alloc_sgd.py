@@ -1,7 +1,8 @@
-"""The allocation-free step with the SGD update, against the oracle, and its
-refusal of a hysteresis it cannot carry (its scaler state has no count).
-Sorts after the first allocation-free test file, which checks the first call's
-device set-up."""
+"""The allocation-free step with the SGD update, against the oracle; its
+refusal of a hysteresis it cannot carry (its scaler state has no count); and
+the step on a shard large enough that the AdamW pass takes chunks from the
+counter in the static scratch.  Sorts after the first allocation-free test
+file, which checks the first call's device set-up."""
 import ctypes
 
 import pytest
@@ -9,8 +10,9 @@ import torch
 
 import oracle
 import synth
-from mixed_precision_zero_b200 import Hparams, NeoxError, _abi
+from mixed_precision_zero_b200 import Hparams, NeoxError, NeoxShard, _abi
 from tests.gpu_harness import oracle_hparams, to_u16
+from tests.test_gpu_chunked import N, SEGS, _equal, _grads, _state
 
 pytestmark = pytest.mark.gpu
 
@@ -60,3 +62,23 @@ def test_noalloc_rejects_hysteresis():
                                      w.data_ptr(), 1e-3, torch.cuda.current_stream().cuda_stream)
     assert ei.value.status == _abi.NEOX_ERR_INVALID_ARGUMENT and "hysteresis" in str(ei.value)
     assert (state.scale, state.good, state.t) == (1024.0, 0, 0)
+
+
+def test_noalloc_step_equals_handle_when_chunked():
+    torch.cuda.set_device(0)
+    hp = Hparams(clip_norm=1.0, init_scale=2.0 ** 12, scale_window=2)
+    a, b = _state(74), _state(74)
+    shard = NeoxShard(a[0], a[1], a[2], hp, segments=SEGS)
+    seg_arr = (_abi.neox_segment * len(SEGS))(*[_abi.neox_segment(o, c, w) for o, c, w in SEGS])
+    desc = _abi.neox_shard_desc(N, _abi.NEOX_FP16, _abi.NEOX_FP16, ctypes.cast(seg_arr, ctypes.POINTER(_abi.neox_segment)),
+                                len(SEGS), 0.0, b[0].data_ptr(), b[1].data_ptr(), b[2].data_ptr(), 1)
+    state = _abi.neox_scaler_state(hp.init_scale, 0, 0)
+    g = torch.empty(N, dtype=torch.float16, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    for s in range(1, 5):
+        _grads(g, s, shard.get_state()[0], 74)
+        ra = shard.step([g], a[3], 1e-3)
+        rb = _abi.neox_shard_step_noalloc(desc, hp.c(), state, [g.data_ptr()], b[3].data_ptr(), 1e-3, stream)
+        assert (ra.overflow, ra.loss_scale_next, ra.applied_steps) == (rb.overflow, rb.loss_scale_next, rb.applied_steps)
+    _equal(a, b)
+    shard.close()
