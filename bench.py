@@ -18,6 +18,7 @@ Prints one JSON line (rank 0).
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import os
@@ -496,23 +497,60 @@ def run_b200(args):
     except Exception as exc:  # reported, not fatal: the headline is the synchronous call
         graph_line = {"error": f"{type(exc).__name__}: {exc}"}
 
-    # end to end through the public API: grads from pinned host memory each step
+    # End to end through the public API: every step copies its gradients from
+    # pinned host memory and reads its result back.  One rank: the gradients
+    # are double-buffered, so the copy for step s + 1 (on a copy stream)
+    # overlaps step s (neox_shard_step_async, whose result the GPU writes into
+    # pinned host memory).  Several ranks: the split step, one after the other.
     host_grads = [g.cpu().pin_memory() for g in grads]
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if ws > 1:
         dist.barrier()
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
-        for g, hg in zip(grads, host_grads):
-            g.copy_(hg, non_blocking=True)
-        res = shard.step(grads, params, wl.lr)
-    e1.record(stream)
-    torch.cuda.synchronize()
+    applied0 = shard.get_state()[2]
+    if not split:
+        from mixed_precision_zero_b200 import _abi
+        bufs = [grads, [torch.empty_like(g) for g in grads]]
+        res_host = [torch.zeros(64, dtype=torch.uint8).pin_memory() for _ in range(2)]
+        copy_stream = torch.cuda.Stream(device=dev)
+        copied = [torch.cuda.Event() for _ in range(2)]
+        done = [torch.cuda.Event() for _ in range(2)]
+        nres = ctypes.sizeof(_abi.neox_step_result)
+        e2e_results = []
+        e0.record(stream)
+        for s in range(args.e2e_steps):
+            j = s % 2
+            with torch.cuda.stream(copy_stream):
+                if s >= 2:
+                    copy_stream.wait_event(done[j])  # step s - 2 has finished reading buffer j
+                for b, hg in zip(bufs[j], host_grads):
+                    b.copy_(hg, non_blocking=True)
+                copied[j].record(copy_stream)
+            stream.wait_event(copied[j])
+            shard.step_async(bufs[j], params, wl.lr, result=res_host[j], stream=stream)
+            done[j].record(stream)
+            if s >= 1:  # the previous step's result, read on the host while this step runs
+                done[1 - j].synchronize()
+                e2e_results.append(_abi.neox_step_result.from_buffer_copy(res_host[1 - j].numpy().tobytes()[:nres]))
+        done[(args.e2e_steps - 1) % 2].synchronize()
+        e2e_results.append(_abi.neox_step_result.from_buffer_copy(
+            res_host[(args.e2e_steps - 1) % 2].numpy().tobytes()[:nres]))
+        e1.record(stream)
+        torch.cuda.synchronize()
+        assert [r.applied_steps for r in e2e_results] == list(range(applied0 + 1, applied0 + args.e2e_steps + 1))
+        d2h = nres  # the result record the GPU writes into pinned host memory each step
+    else:
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            for g, hg in zip(grads, host_grads):
+                g.copy_(hg, non_blocking=True)
+            res = one_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        d2h = 64  # the step's device scalar block, read into pinned memory by every call
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     e2e_value = total_params * args.e2e_steps / (e2e_ms * 1e-3) / 1e9
     h2d = sum(g.numel() * g.element_size() for g in grads)
-    d2h = 64  # the step's device scalar block, read into pinned memory by every call
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
