@@ -21,7 +21,7 @@ constexpr int kMaxGrads = 64;
 constexpr int kThreads1 = 512;   // pass-1 block
 constexpr int kUnroll1 = 4;      // pass-1 vectors in flight per thread
 constexpr int kThreads3 = 256;   // pass-2 block
-constexpr int kChunk3 = 4;       // pass-2 (AdamW) vectors per thread in each dynamically taken chunk
+constexpr int kChunk3 = 2;       // pass-2 (AdamW) vectors per thread in each chunk taken from the counter
 constexpr int kUnrollSgd = 4;    // pass-2 vectors in flight per thread (SGD): measured 6.25 TB/s against 5.83 at 1
 constexpr int kMaxBlocksPerSm = 32;
 

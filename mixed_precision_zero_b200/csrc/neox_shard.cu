@@ -160,7 +160,10 @@ __device__ __forceinline__ void keep_at(SegCursor& cur, unsigned long long i, co
 //    the scalar block (zeroed by pass 1's last block, which this grid waits
 //    for).  Blocks whose memory traffic is served faster take more chunks;
 //    with the static grid-stride the pass that reads the FP32 sum left its
-//    SMs unevenly busy and ran at 5.6 TB/s, against 6.8 with chunks.
+//    SMs unevenly busy and ran at 5.6 TB/s, against 6.8 with chunks.  Chunks
+//    of 2 vectors per thread (64 registers, 4 blocks per SM) measured 6.61
+//    TB/s for the 16-bit-gradient form, against 6.25 with chunks of 4 (69
+//    registers, 3 blocks per SM) and 6.32 for the static grid-stride.
 //    CHUNKED = false (shards of less than one chunk per block, chosen on the
 //    host) keeps the one-vector grid-stride: there a chunk's kChunk3
 //    dependent iterations would be the whole latency.
@@ -408,10 +411,13 @@ cudaError_t launch_pass2(neox_shard* h, const GradPtrs& gp, int K, const float* 
     const bool sgd = h->hp.optimizer == NEOX_SGD, copies = h->wcopies.n > 0;
     auto kern = sgd ? (copies ? sgd_kernel<G, W, VEC, ACC, true> : sgd_kernel<G, W, VEC, ACC, false>)
                     : (copies ? adam_kernel<G, W, VEC, ACC, true, true> : adam_kernel<G, W, VEC, ACC, false, true>);
-    const int grid = grid_for(kern, kThreads3, L.nvec, h->sm_count, 1 << 20);
-    // AdamW takes chunks only when the shard has at least one per block
-    if (!sgd && L.nvec < (unsigned long long)grid * kThreads3 * kChunk3)
+    int grid = grid_for(kern, kThreads3, L.nvec, h->sm_count, 1 << 20);
+    // AdamW takes chunks only when the shard has at least one per block; the
+    // grid-stride instance has its own occupancy, hence its own grid
+    if (!sgd && L.nvec < (unsigned long long)grid * kThreads3 * kChunk3) {
         kern = copies ? adam_kernel<G, W, VEC, ACC, true, false> : adam_kernel<G, W, VEC, ACC, false, false>;
+        grid = grid_for(kern, kThreads3, L.nvec, h->sm_count, 1 << 20);
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kThreads3);

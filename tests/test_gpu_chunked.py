@@ -1,5 +1,5 @@
 """The entry points on shards large enough that the AdamW pass takes its work
-in chunks from the counter in the scalar block (more than 4 x 256 vectors per
+in chunks from the counter in the scalar block (more than 2 x 256 vectors per
 block of its grid).  Each entry point resets or uses that counter its own way:
 the split step (statistics pass, then the decision kernel), the asynchronous
 step replayed from a CUDA graph and the weight copies (their own kernel
