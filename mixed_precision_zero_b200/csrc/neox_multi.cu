@@ -155,73 +155,61 @@ mt_stats_kernel(const MtTensor* __restrict__ tens, int ntensors, const uint16_t*
 }
 
 // ---------------------------------------------------------------- pass 2
-template <bool SGD, class G, class W, int VEC, int KFIX>
-__device__ __forceinline__ void mt_p2_tensor(const GradTab& gp, int K_rt, const MtTensor& T, float keep1, float c,
-                                             float inv_us, const AdamArgs& a) {
+// Pass 2 with plain SGD over one tensor, grid-stride from the tensor's
+// rotated start, kUnrollSgd strides in flight per thread (its loads are too
+// few per vector to cover the memory latency one at a time).
+template <class G, class W, int VEC, int KFIX>
+__device__ __forceinline__ void mt_sgd_tensor(const GradTab& gp, int K_rt, const MtTensor& T, float keep1, float c,
+                                              float inv_us, const AdamArgs& a) {
     const int K = KFIX ? KFIX : K_rt;
     float keep[VEC];
 #pragma unroll
     for (int e = 0; e < VEC; e++) keep[e] = keep1;
     const unsigned long long stride = (unsigned long long)gridDim.x * kMtThreads3;
     float* __restrict__ master = T.master;
-    float* __restrict__ m = T.m;
-    float* __restrict__ v = T.v;
     uint16_t* __restrict__ w = T.w;
     const unsigned long long nvec = T.nvec, head = T.head;
     unsigned long long vi = rotated_start<kMtThreads3>(T.before);
-    if constexpr (SGD) {
-        // kUnrollSgd strides in flight per thread, as in the flat SGD pass
-        // (its loads are too few to cover the memory latency one at a time).
-        constexpr int U = kUnrollSgd;
-        for (; vi + (U - 1) * stride < nvec; vi += U * stride) {
-            float g[U][VEC], p[U][VEC];
-            ingest_batch<G, VEC, U>(gp, K, head + vi * VEC, stride * VEC, a.inv_pre, inv_us, g);
+    constexpr int U = kUnrollSgd;
+    for (; vi + (U - 1) * stride < nvec; vi += U * stride) {
+        float g[U][VEC], p[U][VEC];
+        ingest_batch<G, VEC, U>(gp, K, head + vi * VEC, stride * VEC, a.inv_pre, inv_us, g);
 #pragma unroll
-            for (int u = 0; u < U; u++) ld32<VEC>(master + head + (vi + u * stride) * VEC, p[u]);
+        for (int u = 0; u < U; u++) ld32<VEC>(master + head + (vi + u * stride) * VEC, p[u]);
 #pragma unroll
-            for (int u = 0; u < U; u++) {
-                const unsigned long long i = head + (vi + u * stride) * VEC;
-                sgd_vec<VEC>(g[u], keep, c, a.lr, p[u]);
-                st32<VEC>(master + i, p[u]);
-                st16<W, VEC>(w + i, p[u]);
-            }
+        for (int u = 0; u < U; u++) {
+            const unsigned long long i = head + (vi + u * stride) * VEC;
+            sgd_vec<VEC>(g[u], keep, c, a.lr, p[u]);
+            st32<VEC>(master + i, p[u]);
+            st16<W, VEC>(w + i, p[u]);
         }
     }
     for (; vi < nvec; vi += stride) {
         const unsigned long long i = head + vi * VEC;
-        float g[VEC], p[VEC], mm[VEC], vv[VEC];
+        float g[VEC], p[VEC];
         ingest<G, VEC>(gp, K, i, a.inv_pre, inv_us, g);
         ld32<VEC>(master + i, p);
-        if constexpr (SGD) {
-            sgd_vec<VEC>(g, keep, c, a.lr, p);
-            st32<VEC>(master + i, p);
-        } else {
-            ld32<VEC>(m + i, mm);
-            ld32<VEC>(v + i, vv);
-            adam_vec<VEC>(g, keep, c, a, p, mm, vv);
-            st32<VEC>(master + i, p);
-            st32<VEC>(m + i, mm);
-            st32<VEC>(v + i, vv);
-        }
+        sgd_vec<VEC>(g, keep, c, a.lr, p);
+        st32<VEC>(master + i, p);
         st16<W, VEC>(w + i, p);
     }
 }
 
-template <bool SGD, class G, class W, int KFIX>
-__device__ __forceinline__ void mt_p2_dispatch(const MtTensor& T, const GradTab& gp, int K, float keep1, float c,
-                                               float inv_us, const AdamArgs& a) {
+template <class G, class W, int KFIX>
+__device__ __forceinline__ void mt_sgd_dispatch(const MtTensor& T, const GradTab& gp, int K, float keep1, float c,
+                                                float inv_us, const AdamArgs& a) {
     switch (T.vec) {
-        case 8: mt_p2_tensor<SGD, G, W, 8, KFIX>(gp, K, T, keep1, c, inv_us, a); break;
-        case 4: mt_p2_tensor<SGD, G, W, 4, KFIX>(gp, K, T, keep1, c, inv_us, a); break;
-        case 2: mt_p2_tensor<SGD, G, W, 2, KFIX>(gp, K, T, keep1, c, inv_us, a); break;
-        default: mt_p2_tensor<SGD, G, W, 1, KFIX>(gp, K, T, keep1, c, inv_us, a); break;
+        case 8: mt_sgd_tensor<G, W, 8, KFIX>(gp, K, T, keep1, c, inv_us, a); break;
+        case 4: mt_sgd_tensor<G, W, 4, KFIX>(gp, K, T, keep1, c, inv_us, a); break;
+        case 2: mt_sgd_tensor<G, W, 2, KFIX>(gp, K, T, keep1, c, inv_us, a); break;
+        default: mt_sgd_tensor<G, W, 1, KFIX>(gp, K, T, keep1, c, inv_us, a); break;
     }
 }
 
-// The whole of pass 2 over every tensor, tensor by tensor, each grid-stride
-// (used for SGD; the AdamW pass is mt_adam_chunked_kernel below).
-template <bool SGD, class G, class W>
-__device__ __forceinline__ void mt_update(const MtTensor* __restrict__ tens, int ntensors,
+// Pass 2 with plain SGD over every tensor, tensor by tensor (the AdamW pass
+// is mt_adam_chunked_kernel below).
+template <class G, class W>
+__device__ __forceinline__ void mt_sgd_update(const MtTensor* __restrict__ tens, int ntensors,
                                           const uint16_t* const* __restrict__ gtab, int K, const AdamArgs& a_arg,
                                           const DevScalars* __restrict__ sc) {
     asm volatile("griddepcontrol.wait;" ::: "memory");  // pass 1's results
@@ -246,8 +234,8 @@ __device__ __forceinline__ void mt_update(const MtTensor* __restrict__ tens, int
         if (T.numel == 0) continue;
         const GradTab gp{gtab, T.gbase};
         const float keep1 = __fsub_rn(1.0f, __fmul_rn(a.lr, T.wd));  // fl32(1 - fl32(lr * wd))
-        if (K == 1) mt_p2_dispatch<SGD, G, W, 1>(T, gp, K, keep1, c, inv_us, a);
-        else mt_p2_dispatch<SGD, G, W, 0>(T, gp, K, keep1, c, inv_us, a);
+        if (K == 1) mt_sgd_dispatch<G, W, 1>(T, gp, K, keep1, c, inv_us, a);
+        else mt_sgd_dispatch<G, W, 0>(T, gp, K, keep1, c, inv_us, a);
         if ((unsigned)ti % gridDim.x == blockIdx.x) {  // this tensor's head and tail
             const unsigned long long tail0 = T.head + T.nvec * T.vec;
             const unsigned long long extra = T.head + (T.numel - tail0);
@@ -255,14 +243,7 @@ __device__ __forceinline__ void mt_update(const MtTensor* __restrict__ tens, int
                 const unsigned long long i = j < T.head ? j : tail0 + (j - T.head);
                 float g[1], p[1] = {T.master[i]}, keep[1] = {keep1};
                 ingest<G, 1>(gp, K, i, a.inv_pre, inv_us, g);
-                if constexpr (SGD) {
-                    sgd_vec<1>(g, keep, c, a.lr, p);
-                } else {
-                    float mm[1] = {T.m[i]}, vv[1] = {T.v[i]};
-                    adam_vec<1>(g, keep, c, a, p, mm, vv);
-                    T.m[i] = mm[0];
-                    T.v[i] = vv[0];
-                }
+                sgd_vec<1>(g, keep, c, a.lr, p);
                 T.master[i] = p[0];
                 T.w[i] = W::enc(p[0]);
             }
@@ -379,7 +360,7 @@ template <class G, class W>
 __global__ void __launch_bounds__(kMtThreads3)
 mt_sgd_kernel(const MtTensor* __restrict__ tens, int ntensors, const uint16_t* const* __restrict__ gtab, int K,
               AdamArgs a, const DevScalars* __restrict__ sc) {
-    mt_update<true, G, W>(tens, ntensors, gtab, K, a, sc);
+    mt_sgd_update<G, W>(tens, ntensors, gtab, K, a, sc);
 }
 
 using MtSgdKernel = void (*)(const MtTensor*, int, const uint16_t* const*, int, AdamArgs, const DevScalars*);
