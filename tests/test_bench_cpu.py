@@ -1,0 +1,38 @@
+"""bench.py's bookkeeping on CPU: the algorithmic bytes the roofline divides
+by, and the source hash that ties recorded ncu counters to the kernel code."""
+import os
+import shutil
+
+import bench
+
+
+def test_algorithmic_bytes_per_parameter():
+    # AdamW, one 16-bit buffer: pass 1 reads the gradient; pass 2 reads it again
+    # with master/m/v and writes master/m/v and the 16-bit weight
+    assert bench.alg_bytes_per_param(1, False) == (2, 2 + 12 + 12 + 2)
+    # eight buffers through the FP32 sum: pass 1 writes it, pass 2 reads it instead
+    assert bench.alg_bytes_per_param(8, True) == (16 + 4, 4 + 12 + 12 + 2)
+    # SGD leaves m and v alone
+    assert bench.alg_bytes_per_param(1, False, sgd=True) == (2, 2 + 4 + 4 + 2)
+    assert sum(bench.alg_bytes_per_param(1, False)) == 30
+
+
+def test_source_hash_ignores_comments_but_not_code(tmp_path):
+    copies = []
+    for src in bench.KERNEL_SRCS:
+        dst = tmp_path / os.path.basename(src)
+        shutil.copy(src, dst)
+        copies.append(str(dst))
+    orig = bench.KERNEL_SRCS
+    try:
+        bench.KERNEL_SRCS = copies
+        h0 = bench.kernel_source_hash()
+        assert h0 == bench.kernel_source_hash() and len(h0) == 16
+        with open(copies[0], "a") as f:
+            f.write("\n// a comment\n/* a block\n   comment */\n\n   \n")
+        assert bench.kernel_source_hash() == h0
+        with open(copies[0], "a") as f:
+            f.write("static int g_extra_symbol = 1;\n")
+        assert bench.kernel_source_hash() != h0
+    finally:
+        bench.KERNEL_SRCS = orig
