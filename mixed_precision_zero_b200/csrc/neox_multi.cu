@@ -11,14 +11,17 @@
 // shards model state across ranks, Adam state FP32, weights FP16, dynamic
 // loss scaling, gradient pre-divide and clipping.
 //
-// Work decomposition: both kernels walk the tensors in order and cover each
-// tensor grid-stride across the whole grid, exactly as the flat kernels cover
-// the flat shard (an outer loop over tensors; no synchronisation between
-// tensors).  Each tensor keeps its own vector width and peeled head, chosen
-// from its own pointers; its head and ragged tail are done by block
-// (tensor index mod grid).  A per-block chunk decomposition was measured 11%
-// slower: every block then streams its own distant region instead of all
-// warps streaming one window together.
+// Work decomposition.  Each tensor keeps its own vector width and peeled
+// head, chosen from its own pointers; its head and ragged tail are done by
+// block (tensor index mod grid).
+//  * Pass 1 and the SGD pass walk the tensors in order and cover each one
+//    grid-stride across the whole grid, starting where the previous tensor
+//    left off (no synchronisation between tensors).
+//  * The AdamW pass treats the vectors of all tensors as one sequence and
+//    hands it out in chunks from the counter in the scalar block, as the flat
+//    pass does.
+// A static decomposition into per-block chunks (every block streaming its own
+// distant region) was measured 11% slower than the grid-stride.
 
 #include "neox_shard.h"
 #include "neox_common.cuh"
@@ -222,9 +225,9 @@ __device__ __forceinline__ void mt_sgd_update(const MtTensor* __restrict__ tens,
         a.step_size = sc->step_size;
         a.bcs = sc->bc2_sqrt;
     }
-    // Descriptors are staged in the dynamic shared memory, whose size (set at
-    // launch) also holds the kernel to 3 blocks per SM: a measured 4% better
-    // for this read/write stream than the 4 blocks its registers would allow.
+    // Descriptors are staged in dynamic shared memory, kMtDescBatch3 at a time,
+    // so that a warp reads each tensor's pointers from shared memory instead of
+    // waiting on a dependent global load at every tensor boundary.
     extern __shared__ MtTensor tsh_dyn[];
     for (int base = 0; base < ntensors; base += kMtDescBatch3) {
     const int cnt = ntensors - base < kMtDescBatch3 ? ntensors - base : kMtDescBatch3;
