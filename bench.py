@@ -363,6 +363,9 @@ def run_multi(args):
     for _ in range(args.warmup):
         multi.step(wl.lr)
     t0 = multi.get_state()[2]
+    multi.reset_profile()
+    multi.set_profiling(True)
+    launches0 = multi.profile().launches
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     with ClockSampler(0) as clocks:
@@ -373,8 +376,12 @@ def run_multi(args):
         torch.cuda.synchronize()
     assert multi.get_state()[2] - t0 == args.steps
     ms = e0.elapsed_time(e1)
+    prof = multi.profile()
+    multi.set_profiling(False)
     p1b, p2b = alg_bytes_per_param(wl.K, False, args.optimizer == "sgd")
     peak, kind = hbm_peak()
+    p2_ms = prof.update_pass_ms / prof.steps
+    kernel2 = "mt_sgd_kernel" if args.optimizer == "sgd" else "mt_adam_chunked_kernel"
     line = {"metric": METRIC_SGD if args.optimizer == "sgd" else METRIC, "value": wl.numel * args.steps / (ms * 1e-3) / 1e9, "unit": UNIT, "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "impl": "b200",
@@ -383,6 +390,12 @@ def run_multi(args):
             "hbm": {"step_gbs": (p1b + p2b) * wl.numel / (ms / args.steps * 1e-3) / 1e9,
                     "step_frac": (p1b + p2b) * wl.numel / (ms / args.steps * 1e-3) / 1e9 / peak, "peak_gbs": peak,
                     "peak_kind": kind},
+            "roofline": {"bound": "hbm", "kernel": f"{kernel2} (pass 2)",
+                         "achieved": p2b * wl.numel / (p2_ms * 1e-3) / 1e9, "peak": peak, "unit": "GB/s",
+                         "frac": p2b * wl.numel / (p2_ms * 1e-3) / 1e9 / peak, "peak_kind": kind, "traffic": None,
+                         "alg_bytes_per_launch": p2b * wl.numel, "avg_launch_ms": p2_ms,
+                         "grad_pass_avg_ms": prof.grad_pass_ms / prof.steps},
+            "gpu_launches": prof.launches - launches0,
             "clocks": clocks.summary()}
     multi.close()
     print(json.dumps(line), flush=True)

@@ -386,6 +386,11 @@ neox_status neox_multi_get_state(const neox_multi* h, float* scale, int32_t* goo
 neox_status neox_multi_set_state(neox_multi* h, float scale, int32_t good, int64_t t);
 neox_status neox_multi_get_hysteresis(const neox_multi* h, int32_t* count);
 neox_status neox_multi_set_hysteresis(neox_multi* h, int32_t count);
+/* Per-pass timing of synchronous steps, as neox_shard_set_profiling /
+ * get_profile / reset_profile (the same neox_profile record). */
+neox_status neox_multi_set_profiling(neox_multi* h, int32_t enable);
+neox_status neox_multi_get_profile(const neox_multi* h, neox_profile* out);
+neox_status neox_multi_reset_profile(neox_multi* h);
 void neox_multi_destroy(neox_multi* h);
 const char* neox_multi_last_error(const neox_multi* h);
 

@@ -27,7 +27,8 @@ from ._abi import (NEOX_BF16, NEOX_ERR_CUDA, NEOX_ERR_INVALID_ARGUMENT, NEOX_ERR
                    neox_multi_set_hparams, neox_multi_destroy, neox_shard_grad_stats, neox_shard_apply,
                    neox_shard_set_weight_copies, neox_shard_get_hysteresis, neox_shard_set_hysteresis,
                    neox_multi_get_hysteresis, neox_multi_set_hysteresis, NEOX_ADAMW, NEOX_SGD,
-                   NEOX_SHARD_ACCUMULATE)
+                   NEOX_SHARD_ACCUMULATE, neox_multi_set_profiling, neox_multi_get_profile,
+                   neox_multi_reset_profile)
 
 __all__ = ["NeoxShard", "NeoxMultiShard", "Hparams", "NeoxError", "neox_shard_create", "neox_shard_step",
            "neox_shard_destroy", "neox_shard_set_hparams", "neox_shard_get_state",
@@ -283,6 +284,15 @@ class NeoxMultiShard:
 
     def get_hysteresis(self) -> int:
         return neox_multi_get_hysteresis(self.handle)
+
+    def set_profiling(self, enable: bool) -> None:
+        neox_multi_set_profiling(self.handle, enable)
+
+    def profile(self) -> neox_profile:
+        return neox_multi_get_profile(self.handle)
+
+    def reset_profile(self) -> None:
+        neox_multi_reset_profile(self.handle)
 
     def set_hysteresis(self, count: int) -> None:
         neox_multi_set_hysteresis(self.handle, count)

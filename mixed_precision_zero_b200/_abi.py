@@ -159,6 +159,12 @@ def lib() -> ctypes.CDLL:
         L.neox_multi_get_state.restype = S
         L.neox_multi_set_state.argtypes = [_H, ctypes.c_float, ctypes.c_int32, ctypes.c_int64]
         L.neox_multi_set_state.restype = S
+        L.neox_multi_set_profiling.argtypes = [_H, ctypes.c_int32]
+        L.neox_multi_set_profiling.restype = S
+        L.neox_multi_get_profile.argtypes = [_H, ctypes.POINTER(neox_profile)]
+        L.neox_multi_get_profile.restype = S
+        L.neox_multi_reset_profile.argtypes = [_H]
+        L.neox_multi_reset_profile.restype = S
         L.neox_multi_get_hysteresis.argtypes = [_H, ctypes.POINTER(ctypes.c_int32)]
         L.neox_multi_get_hysteresis.restype = S
         L.neox_multi_set_hysteresis.argtypes = [_H, ctypes.c_int32]
@@ -377,6 +383,20 @@ def neox_multi_set_hparams(h: int, hp: neox_hparams) -> None:
     st = lib().neox_multi_set_hparams(h, ctypes.byref(hp))
     if st != NEOX_OK:
         raise NeoxError(st, _merr(h))
+
+
+def neox_multi_set_profiling(h: int, enable: bool) -> None:
+    lib().neox_multi_set_profiling(h, int(enable))
+
+
+def neox_multi_get_profile(h: int) -> neox_profile:
+    p = neox_profile()
+    lib().neox_multi_get_profile(h, ctypes.byref(p))
+    return p
+
+
+def neox_multi_reset_profile(h: int) -> None:
+    lib().neox_multi_reset_profile(h)
 
 
 def neox_multi_destroy(h: int) -> None:

@@ -407,6 +407,10 @@ struct neox_multi {
     int* d_part_b = nullptr;
     DevScalars* h_sc = nullptr;
     std::vector<MtTensor> tens;  // host copy (pointers and layouts)
+    // profiling: events around the two passes of synchronous steps
+    bool profiling = false;
+    cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};
+    neox_profile prof{};
     std::string last_error;
 };
 
@@ -431,6 +435,8 @@ void mfree(neox_multi* h) {
     if (h->d_part_s) cudaFree(h->d_part_s);
     if (h->d_part_b) cudaFree(h->d_part_b);
     if (h->h_sc) cudaFreeHost(h->h_sc);
+    for (auto& ev : h->ev)
+        if (ev) cudaEventDestroy(ev);
 }
 
 // Pointer table and layout of every tensor; returns an error message or "".
@@ -486,7 +492,7 @@ int mt_grid(Kern kernel, int threads, unsigned long long total_vecs, int sm_coun
 }
 
 neox_status mt_enqueue(neox_multi* h, float lr, const float* lr_dev, cudaStream_t st, bool device_bc,
-                       neox_step_result* result) {
+                       neox_step_result* result, bool timed = false) {
     if (!lr_dev && (!finite(lr) || lr < 0.0f)) return mfail(h, NEOX_ERR_INVALID_ARGUMENT, "lr must be finite and >= 0");
     if (result && ((uintptr_t)result & 7u)) return mfail(h, NEOX_ERR_INVALID_ARGUMENT, "result must be 8-byte aligned");
     if (lr_dev && ((uintptr_t)lr_dev & 3u)) return mfail(h, NEOX_ERR_INVALID_ARGUMENT, "lr_device must be 4-byte aligned");
@@ -497,13 +503,16 @@ neox_status mt_enqueue(neox_multi* h, float lr, const float* lr_dev, cudaStream_
     sa.result = result;
 
     cudaError_t e;
+    if (timed && (e = cudaEventRecord(h->ev[0], st)) != cudaSuccess) return mcuda_fail(h, e, "cudaEventRecord");
     {
         auto k1 = h->gdtype == NEOX_FP16 ? mt_stats_kernel<F16> : mt_stats_kernel<BF16>;
         const int grid = h->grid1;
         k1<<<grid, kMtThreads1, 0, st>>>(h->d_tens, h->ntensors, h->d_gtab, h->K, sa, h->d_part_s, h->d_part_b,
                                          h->d_sc);
         if ((e = cudaGetLastError()) != cudaSuccess) return mcuda_fail(h, e, "pass-1 launch");
+        h->prof.launches += 1;
     }
+    if (timed && (e = cudaEventRecord(h->ev[1], st)) != cudaSuccess) return mcuda_fail(h, e, "cudaEventRecord");
     if (h->numel > 0) {
         const bool sgd = h->hp.optimizer == NEOX_SGD;
         cudaLaunchConfig_t cfg = {};
@@ -528,7 +537,9 @@ neox_status mt_enqueue(neox_multi* h, float lr, const float* lr_dev, cudaStream_
                                    total);
         }
         if (e != cudaSuccess) return mcuda_fail(h, e, "pass-2 launch");
+        h->prof.launches += 1;
     }
+    if (timed && (e = cudaEventRecord(h->ev[2], st)) != cudaSuccess) return mcuda_fail(h, e, "cudaEventRecord");
     return NEOX_OK;
 }
 
@@ -601,7 +612,9 @@ neox_status neox_multi_create(const neox_tensor_set* set, const neox_hparams* hp
             (e = cudaMalloc(&h->d_sc, sizeof(DevScalars))) != cudaSuccess ||
             (e = cudaMalloc(&h->d_part_s, sizeof(double) * h->max_parts)) != cudaSuccess ||
             (e = cudaMalloc(&h->d_part_b, sizeof(int) * h->max_parts)) != cudaSuccess ||
-            (e = cudaMallocHost(&h->h_sc, sizeof(DevScalars))) != cudaSuccess) {
+            (e = cudaMallocHost(&h->h_sc, sizeof(DevScalars))) != cudaSuccess ||
+            (e = cudaEventCreate(&h->ev[0])) != cudaSuccess || (e = cudaEventCreate(&h->ev[1])) != cudaSuccess ||
+            (e = cudaEventCreate(&h->ev[2])) != cudaSuccess) {
             st = mcuda_fail(nullptr, e, "allocation");
             goto done;
         }
@@ -706,7 +719,7 @@ neox_status neox_multi_step(neox_multi* h, float lr, void* cuda_stream, neox_ste
     DeviceGuard g(h->device);
     if (!g.ok) return mfail(h, NEOX_ERR_CUDA, "cudaSetDevice failed");
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
-    if (neox_status s = mt_enqueue(h, lr, nullptr, st, h->async_used, nullptr); s != NEOX_OK) return s;
+    if (neox_status s = mt_enqueue(h, lr, nullptr, st, h->async_used, nullptr, h->profiling); s != NEOX_OK) return s;
     cudaError_t e;
     if ((e = cudaMemcpyAsync(h->h_sc, h->d_sc, sizeof(DevScalars), cudaMemcpyDeviceToHost, st)) != cudaSuccess)
         return mcuda_fail(h, e, "cudaMemcpyAsync result");
@@ -722,6 +735,36 @@ neox_status neox_multi_step(neox_multi* h, float lr, void* cuda_stream, neox_ste
     h->scale = r.scale;
     h->good = r.good;
     h->t = r.t;
+    if (h->profiling) {
+        float t01 = 0.f, t12 = 0.f;
+        cudaEventElapsedTime(&t01, h->ev[0], h->ev[1]);
+        cudaEventElapsedTime(&t12, h->ev[1], h->ev[2]);
+        h->prof.steps += 1;
+        h->prof.grad_pass_ms += t01;
+        h->prof.update_pass_ms += t12;
+        h->prof.last_grad_pass_ms = t01;
+        h->prof.last_update_pass_ms = t12;
+    }
+    return NEOX_OK;
+}
+
+neox_status neox_multi_set_profiling(neox_multi* h, int32_t enable) {
+    if (!h) return NEOX_ERR_INVALID_ARGUMENT;
+    h->profiling = enable != 0;
+    return NEOX_OK;
+}
+
+neox_status neox_multi_get_profile(const neox_multi* h, neox_profile* out) {
+    if (!h || !out) return NEOX_ERR_INVALID_ARGUMENT;
+    *out = h->prof;
+    return NEOX_OK;
+}
+
+neox_status neox_multi_reset_profile(neox_multi* h) {
+    if (!h) return NEOX_ERR_INVALID_ARGUMENT;
+    const int64_t launches = h->prof.launches;
+    h->prof = neox_profile{};
+    h->prof.launches = launches;
     return NEOX_OK;
 }
 
