@@ -1,14 +1,16 @@
 #!/usr/bin/env python
 """Benchmark of the per-rank mixed-precision Adam shard step on B200.
 
-    python bench.py [--gpus N --steps K --warmup W] [--workload pythia_1p4b]
+    python bench.py [--gpus N --steps K --warmup W] [--workload opt_5b]
     python bench.py --impl reference ...      # the CPU oracle as the reference arm
 
 One step = one neox_shard_step call over the whole owned shard: pass 1 (ingest,
 overflow flag, global norm, loss scaler, clip coefficient) and pass 2 (AdamW on
-FP32 master/m/v + cast to the 16-bit working copy).  Inputs are resident in HBM
-(22.6 GB for the default 1.41e9-parameter shard, far above the 126 MB L2, so no
-flush is needed between steps).  Under torchrun every rank steps its own shard of
+FP32 master/m/v + cast to the 16-bit working copy).  The default workload is the
+largest single-GPU one, the OPT-style 5e9-parameter BF16 shard; the others
+(``--workload pythia_1p4b``, ``neox20b_slice``, ``accum8``, ``tiny``) run the
+same way.  Inputs are resident in HBM (80 GB for the default shard, far above
+the 126 MB L2, so no flush is needed between steps).  Under torchrun every rank steps its own shard of
 the same size (weak scaling) with the split step: pass 1, a 16-byte NCCL
 all-reduce of {sum of squares, non-finite flag}, then the shared decision and
 pass 2, as data-parallel ranks with one global norm and loss scale do.
@@ -49,7 +51,7 @@ def parse_args(argv=None):
     p.add_argument("--steps", type=int, default=100)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["b200", "reference"], default="b200")
-    p.add_argument("--workload", default="pythia_1p4b")
+    p.add_argument("--workload", default="opt_5b")
     p.add_argument("--e2e-steps", type=int, default=5)
     p.add_argument("--split", action="store_true",
                    help="run the split step (statistics, all-reduce, apply) even on one rank")

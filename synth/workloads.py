@@ -121,6 +121,14 @@ def pythia_2layer() -> Workload:
     return pythia_1p4b(layers=2)
 
 
+def opt_5b_cut() -> Workload:
+    """The OPT-style recipe at 2^28 parameters (4.8 GB on the device): the BF16
+    kernel instances of the 5e9-element shard at a size that detailed profiler
+    captures handle."""
+    import dataclasses
+    return dataclasses.replace(opt_style_5b(numel=1 << 28), name="opt_style_bf16_2e28")
+
+
 def accum8_small() -> Workload:
     """The 8-buffer recipe at 2^26 parameters (2.4 GB on the device with the
     FP32 sum buffer): a size that detailed profiler captures handle."""
@@ -130,4 +138,4 @@ def accum8_small() -> Workload:
 
 ALL = {"tiny": tiny, "pythia_1p4b": pythia_1p4b, "neox20b_slice": neox20b_zero1_slice,
        "accum8": accum8_predivide, "opt_5b": opt_style_5b, "pythia_2layer": pythia_2layer,
-       "accum8_small": accum8_small}
+       "accum8_small": accum8_small, "opt_5b_cut": opt_5b_cut}
