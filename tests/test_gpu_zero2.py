@@ -11,9 +11,14 @@ maps the other's buffers; then per step:
   - pass 2 updates the slice and stores the cast into every rank's weight
     buffer (the all-gather fused with the cast).
 The result must equal the oracle over the whole model with the K = 2 rank
-gradients as its buffers: bit-exact with clipping off.  The processes
-synchronise only on the host (barriers between steps); no kernel waits on
-another."""
+gradients as its buffers: bit-exact with clipping off.
+
+The ranks are ordered against each other only by zero.zero2_step's stream
+barriers (interprocess CUDA events over this gloo group): there is no device
+synchronisation and no host barrier between the steps, and each rank writes
+its next gradients right after its step returns.  No kernel waits on
+another: the barriers are stream waits on events whose records were issued
+before the waits."""
 import os
 import socket
 import traceback
@@ -46,7 +51,7 @@ def _rank_main(rank, world, port, q, cfg):
         import synth
         from mixed_precision_zero_b200 import Hparams, NeoxShard
         from mixed_precision_zero_b200.peer import PeerMap, allgather_weight_dsts, zero2_grad_ptrs
-        from mixed_precision_zero_b200.zero import zero_step
+        from mixed_precision_zero_b200.zero import make_stream_barrier, zero2_step
         torch.cuda.set_device(0)
         n, steps, lr = cfg["n"], cfg["steps"], cfg["lr"]
         N = world * n
@@ -64,19 +69,21 @@ def _rank_main(rank, world, port, q, cfg):
         shard.set_weight_copies(allgather_weight_dsts(wmap, n))
         gptrs = zero2_grad_ptrs(gmap, n)
         stats = torch.zeros(2, dtype=torch.float64, device="cuda")
+        barrier = make_stream_barrier()
         out = {"host_grads": [], "results": []}
         if rank == 0:
             out["master0"] = master_full.cpu().numpy()
         for s in range(1, steps + 1):
+            # this rank's gradients of step s, written on its stream right after
+            # its previous step returned (no host or device synchronisation)
             synth.gpu_grad_normal16(grads_full, 1e-3, shard.get_state()[0], 7, rank, s)
             if s == cfg["overflow_step"] and rank == 1:
                 grads_full.view(torch.int16)[5] = 0x7C00       # in slice 0: rank 0's pass 1 must see it
-            torch.cuda.synchronize()
+            # barrier, pass 1 over both ranks' copies, all-reduce, pass 2 with the
+            # weight copies, barrier
+            res = zero2_step(shard, gptrs, params, lr, stats, barrier)
+            # read back for the oracle (the step only reads the gradients)
             out["host_grads"].append(grads_full.view(torch.int16).cpu().numpy().view(np.uint16).copy())
-            dist.barrier()                                     # every rank's gradients are written
-            res = zero_step(shard, gptrs, params, lr, stats)     # pass 1, all-reduce, pass 2
-            torch.cuda.synchronize()
-            dist.barrier()                                     # every rank is done reading and storing
             out["results"].append((res.overflow, res.loss_scale_next, res.applied_steps, res.grad_norm))
         out["master"] = master.cpu().numpy()
         out["m"] = m.cpu().numpy()
