@@ -150,6 +150,10 @@ class ShardCase:
         for name, a, b in (("master", gm, self.orc.master), ("m", gmm, self.orc.m), ("v", gv, self.orc.v)):
             check_close(name, a, b)
         check_ulp16(gw, self.orc.w)
+        # non-gating: how far m and v are in FP32 ulps where the absolute floor
+        # would hide a difference (|x| > 1e-30)
+        print(f"max FP32 ulp distance: m {ulp_distance_above(gmm, self.orc.m)}, "
+              f"v {ulp_distance_above(gv, self.orc.v)}")
 
     def guards_intact(self):
         return all(x.guards_intact() for x in (*self.g, self.w, self.master, self.m, self.v))
@@ -169,6 +173,15 @@ def check_close(name, a, b, rtol=1e-5, atol=1e-7):
 def check_ulp16(a, b):
     d = np.abs(ordered16(a) - ordered16(b))
     assert d.max(initial=0) <= 1, f"16-bit weights differ by up to {d.max()} ulp at {np.flatnonzero(d > 1)[:5]}"
+
+
+def ulp_distance_above(a, b, floor=1e-30) -> int:
+    """ulp_distance32 over the elements whose reference b exceeds `floor` in
+    magnitude (a diagnostic of m and v, whose values sit far below the
+    absolute floor of the tolerance)."""
+    b = np.asarray(b, np.float32)
+    sel = np.abs(b) > floor
+    return ulp_distance32(np.asarray(a, np.float32)[sel], b[sel]) if sel.any() else 0
 
 
 def ulp_distance32(a, b) -> int:
