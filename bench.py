@@ -51,7 +51,8 @@ def parse_args(argv=None):
     p.add_argument("--steps", type=int, default=100)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["b200", "reference"], default="b200")
-    p.add_argument("--workload", default="opt_5b")
+    p.add_argument("--workload", default=None,
+                   help="default: opt_5b (the largest single-GPU shard); pythia_1p4b with --zero2")
     p.add_argument("--e2e-steps", type=int, default=5)
     p.add_argument("--split", action="store_true",
                    help="run the split step (statistics, all-reduce, apply) even on one rank")
@@ -61,9 +62,14 @@ def parse_args(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--optimizer", choices=["adamw", "sgd"], default="adamw",
                    help="update rule of pass 2 (sgd: plain SGD, m and v untouched)")
+    p.add_argument("--zero2", action="store_true",
+                   help="ZeRO-2 over peer memory: every rank owns 1/N of the model, pass 1 reads every rank's "
+                        "gradient slice, pass 2 stores the cast into every rank's weight buffer")
     a = p.parse_args(argv)
     if a.warmup < 3:
         p.error("--warmup must be >= 3")
+    if a.workload is None:
+        a.workload = "pythia_1p4b" if a.zero2 else "opt_5b"
     return a
 
 
@@ -233,16 +239,63 @@ def sample_segments(wl, lo, n):
     return segs, inits
 
 
-def run_oracle_sample(wl, n_sample, steps, seconds, rank_seed=0, optimizer="adamw"):
-    """Time the single-threaded oracle on `steps` calls over a contiguous sample
-    of the workload (inputs drawn by the numpy twin of the generator, untimed)."""
-    import numpy as np
+def host_cores() -> int:
+    return max(1, len(os.sched_getaffinity(0)))
 
-    import oracle
+
+def parallel_gen(fn, n, threads, chunk=1 << 22, **kw):
+    """A numpy-twin input array of n elements drawn in contiguous chunks on
+    `threads` host threads (the generators take the first element's index)."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    import numpy as np
+    starts = list(range(0, n, chunk))
+    lo0 = kw.pop("start", 0)
+    with ThreadPoolExecutor(threads) as ex:
+        parts = list(ex.map(lambda a: fn(min(chunk, n - a), start=lo0 + a, **kw), starts))
+    return np.concatenate(parts) if parts else np.zeros(0)
+
+
+def sample_inputs_host(wl, n_sample, threads, rank_seed=0):
+    """A contiguous sample of the workload drawn by the numpy twin of the
+    generator: (lo, master, grads)."""
     import synth
     lo, n = cpu_sample_range(wl, n_sample)
+    master = parallel_gen(synth.master_normal, n, threads, sigma=wl.master_sigma, seed=wl.seed + rank_seed,
+                          tensor_id=0, start=lo)
+    scale = wl.bench_scale or wl.init_scale
+    grads = []
+    for k in range(wl.K):
+        if wl.grad_dist == "t3":
+            grads.append(parallel_gen(synth.grad_t3_16, n, threads, scale=scale, seed=wl.seed + rank_seed,
+                                      tensor_id=k, step=1, bf16=wl.bf16, start=lo))
+        else:
+            grads.append(parallel_gen(synth.grad_normal16, n, threads, sigma=wl.grad_sigma, scale=scale,
+                                      seed=wl.seed + rank_seed, tensor_id=k, step=1, bf16=wl.bf16, start=lo))
+    return lo, master, grads
+
+
+def sample_inputs_device(wl, n_sample, master_dev, grads_dev):
+    """The same kind of sample copied from the workload resident on the GPU
+    (its bytes come from the CUDA twin of the generator): (lo, master, grads)."""
+    import numpy as np
+    import torch
+    lo, n = cpu_sample_range(wl, n_sample)
+    master = master_dev[lo:lo + n].cpu().numpy().copy()
+    grads = [g[lo:lo + n].view(torch.int16).cpu().numpy().view(np.uint16).copy() for g in grads_dev]
+    return lo, master, grads
+
+
+def run_oracle_sample(wl, inputs, steps, seconds, threads=1, optimizer="adamw"):
+    """Time the oracle on up to `steps` calls (stopping once `seconds` have
+    passed) over a contiguous sample of the workload, single-threaded or split
+    over `threads` host threads by contiguous ranges.  The inputs are drawn
+    before, untimed."""
+    import oracle
+    lo, master, grads = inputs
+    n = master.size
     segs, inits = sample_segments(wl, lo, n)
-    master = synth.master_normal(n, wl.master_sigma, wl.seed + rank_seed, 0, start=lo)
+    master = master.astype("float32", copy=True)
     for init, a, c in inits:
         if init == "zero":
             master[a:a + c] = 0
@@ -251,21 +304,19 @@ def run_oracle_sample(wl, n_sample, steps, seconds, rank_seed=0, optimizer="adam
     hp = oracle.OracleHparams(wl.beta1, wl.beta2, wl.eps, wl.clip, wl.predivide, wl.bench_scale or wl.init_scale,
                               2.0, 1.0, wl.scale_window, optimizer=1 if optimizer == "sgd" else 0)
     sh = oracle.OracleShard(master, hp, wbf16=wl.bf16, gbf16=wl.bf16, segments=segs, default_wd=wl.weight_decay)
-    grads = []
-    for k in range(wl.K):
-        if wl.grad_dist == "t3":
-            grads.append(synth.grad_t3_16(n, sh.scale, wl.seed + rank_seed, k, 1, wl.bf16, start=lo))
-        else:
-            grads.append(synth.grad_normal16(n, wl.grad_sigma, sh.scale, wl.seed + rank_seed, k, 1, wl.bf16, start=lo))
+    chunk = max(1 << 16, -(-n // (4 * threads)))   # a few contiguous ranges per thread
     times = []
     t_all = time.perf_counter()
-    for s in range(steps):
+    for _ in range(steps):
         t0 = time.perf_counter()
-        sh.step(grads, wl.lr)
+        if threads > 1:
+            sh.step_threaded(grads, wl.lr, threads, chunk=chunk)
+        else:
+            sh.step(grads, wl.lr)
         times.append(time.perf_counter() - t0)
-        if seconds and time.perf_counter() - t_all > seconds and s >= 0:
+        if seconds and time.perf_counter() - t_all > seconds:
             break
-    return {"n": n, "lo": lo, "times": times}
+    return {"n": n, "lo": lo, "times": times, "threads": threads}
 
 
 # ------------------------------------------------------------------ reference arm
@@ -277,9 +328,12 @@ def run_reference(args):
         return 0
     wl = W.ALL[args.workload]()
     total = args.steps + args.warmup
-    per_step_budget = max(0.2, 150.0 / total)           # whole run within a few minutes
-    n_sample = int(min(1 << 24, max(1 << 16, per_step_budget / 60e-9)))
-    out = run_oracle_sample(wl, n_sample, total, 0.0, optimizer=args.optimizer)
+    cores = host_cores()
+    per_step_budget = max(0.2, 120.0 / total)           # whole run within a few minutes
+    # about 40 ns per element and thread for the AdamW step
+    n_sample = int(min(1 << 27, wl.numel, max(1 << 16, per_step_budget * cores / 40e-9)))
+    inputs = sample_inputs_host(wl, n_sample, cores)
+    out = run_oracle_sample(wl, inputs, total, 0.0, threads=cores, optimizer=args.optimizer)
     times = out["times"][args.warmup:]
     sec = sum(times)
     value = out["n"] * len(times) / sec / 1e9
@@ -289,8 +343,9 @@ def run_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": wl.name, "numel": wl.numel, "grad_buffers": wl.K, "optimizer": args.optimizer,
                    "sample": f"{out['n']} contiguous elements from index {out['lo']} per step"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": f"{out['n']} contiguous elements of {wl.name}, {len(times)} timed steps"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{out['n']} contiguous elements of {wl.name}, {len(times)} timed steps, "
+                                   f"split over {cores} host threads by contiguous ranges"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -567,13 +622,24 @@ def run_b200(args):
     e2e_value = total_params * args.e2e_steps / (e2e_ms * 1e-3) / 1e9
     h2d = sum(g.numel() * g.element_size() for g in grads)
 
-    cpu = None
+    cpu = cpu1 = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        out = run_oracle_sample(wl, 1 << 25, 50, args.cpu_seconds, optimizer=args.optimizer)
+        # the oracle on every host core (contiguous ranges), then on one, on
+        # slices of the resident workload (the bytes the GPU stepped on)
+        cores = host_cores()
+        master_dev = state[0]
+        out = run_oracle_sample(wl, sample_inputs_device(wl, 1 << 27, master_dev, grads), 50,
+                                args.cpu_seconds, threads=cores, optimizer=args.optimizer)
         sec = sum(out["times"])
-        cpu = {"value": out["n"] * len(out["times"]) / sec / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+        cpu = {"value": out["n"] * len(out["times"]) / sec / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"{len(out['times'])} steps over {out['n']} contiguous elements of {wl.name} "
-                         f"(from index {out['lo']}), single-threaded oracle"}
+                         f"(from index {out['lo']}), split over {cores} host threads by contiguous ranges"}
+        out = run_oracle_sample(wl, sample_inputs_device(wl, 1 << 24, master_dev, grads), 50,
+                                args.cpu_seconds / 3, threads=1, optimizer=args.optimizer)
+        sec = sum(out["times"])
+        cpu1 = {"value": out["n"] * len(out["times"]) / sec / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+                "sample": f"{len(out['times'])} steps over {out['n']} contiguous elements of {wl.name} "
+                          f"(from index {out['lo']}), single-threaded"}
 
     clk = clocks.summary()
     line = {
@@ -595,7 +661,9 @@ def run_b200(args):
                      "traffic": traffic, "alg_bytes_per_launch": p2b * wl.numel,
                      "avg_launch_ms": p2_ms, "grad_pass_avg_ms": p1_ms},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "steps": args.e2e_steps},
+                "steps": args.e2e_steps,
+                # the gradients' host-to-device rate over the timed region: the bound of this line
+                "h2d_gbs": h2d * args.e2e_steps / (e2e_ms * 1e-3) / 1e9},
         "gpu_launches": launches,
         "graph": graph_line,
         "clocks": clk,
@@ -603,9 +671,170 @@ def run_b200(args):
     }
     if cpu:
         line["cpu_baseline"] = cpu
+        line["cpu_baseline_single_thread"] = cpu1
     shard.close()
     if dist.is_initialized():
         dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ ZeRO-2 over peer memory
+
+def zero2_plan(wl, world: int, rank: int) -> dict:
+    """This rank's part of a ZeRO-2 job over the whole workload: its slice
+    [lo, lo + n) of the flat model (equal slices), the slice's segment table,
+    and the bytes of one step that cross NVLink for this rank (pass 1 reads
+    the other ranks' copies of its gradient slice, pass 2 writes its cast into
+    the other ranks' weight buffers)."""
+    N = wl.numel
+    if N % world:
+        raise ValueError(f"{N} parameters do not split into {world} equal slices")
+    n = N // world
+    lo = rank * n
+    segs = None
+    if wl.segments:
+        segs = []
+        for off, cnt, wd, _ in wl.segments:
+            a, b = max(off, lo), min(off + cnt, lo + n)
+            if a < b:
+                segs.append((a - lo, b - a, wd))
+    return {"N": N, "n": n, "lo": lo, "segments": segs,
+            "nvlink_read_bytes": (world - 1) * 2 * n, "nvlink_write_bytes": (world - 1) * 2 * n}
+
+
+def run_zero2(args):
+    """The whole-model ZeRO-2 step: N ranks (one per GPU of the node), each the
+    owner of 1/N of the flat model with its FP32 master/m/v, each holding the
+    full gradient of its own micro-batches and a full 16-bit weight copy.  Per
+    step (zero.zero2_step): a stream barrier, pass 1 over the N ranks' copies
+    of the owned gradient slice through CUDA IPC (pre-divide N, FP32 sum kept
+    for pass 2), the 16-byte statistics all-reduce, pass 2 storing the cast
+    into every rank's weight buffer, a stream barrier.  Total work is fixed
+    (one model), so the scaling is strong."""
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    from mixed_precision_zero_b200 import Hparams, NeoxShard
+    from mixed_precision_zero_b200.peer import PeerMap, allgather_weight_dsts, zero2_grad_ptrs
+    from mixed_precision_zero_b200.zero import make_stream_barrier, zero2_step
+    from synth import workloads as W
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    own_group = False
+    if not dist.is_initialized():
+        from datetime import timedelta
+        if "MASTER_ADDR" not in os.environ:  # one rank without torchrun
+            import socket
+            sk = socket.socket()
+            sk.bind(("127.0.0.1", 0))
+            os.environ["MASTER_ADDR"], os.environ["MASTER_PORT"] = "127.0.0.1", str(sk.getsockname()[1])
+            sk.close()
+            os.environ.setdefault("RANK", "0")
+            os.environ.setdefault("WORLD_SIZE", "1")
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+        own_group = True
+    wl = W.ALL[args.workload]()
+    plan = zero2_plan(wl, ws, rank)
+    N, n, lo = plan["N"], plan["n"], plan["lo"]
+    dt = torch.bfloat16 if wl.bf16 else torch.float16
+    scale = wl.bench_scale or wl.init_scale
+    master_full = torch.empty(N, dtype=torch.float32, device=dev)
+    synth.gpu_master_normal(master_full, wl.master_sigma, wl.seed)       # the same model on every rank
+    for s_off, cnt, _, init in (wl.segments or []):
+        if init == "zero":
+            master_full[s_off:s_off + cnt].zero_()
+        elif init == "one":
+            master_full[s_off:s_off + cnt].fill_(1.0)
+    wfull = master_full.to(dt)
+    master = master_full[lo:lo + n].clone()
+    del master_full
+    m, v = torch.zeros_like(master), torch.zeros_like(master)
+    grads_full = torch.empty(N, dtype=dt, device=dev)
+    synth.gpu_grad_normal16(grads_full, wl.grad_sigma, scale, wl.seed + 1000 * rank, 0, 1, wl.bf16)
+    torch.cuda.synchronize()
+    gmap = PeerMap.from_group(grads_full)
+    wmap = PeerMap.from_group(wfull)
+    hp = Hparams(wl.beta1, wl.beta2, wl.eps, wl.clip, float(ws), scale, 2.0, 1.0, wl.scale_window)
+    shard = NeoxShard(master, m, v, hp, wdtype=dt, gdtype=dt, segments=plan["segments"],
+                      weight_decay=wl.weight_decay, max_grads=ws, accumulate=True)
+    params = wfull[lo:lo + n]
+    shard.set_weight_copies(allgather_weight_dsts(wmap, n, wfull.element_size()))
+    gptrs = zero2_grad_ptrs(gmap, n, grads_full.element_size())
+    stats = torch.zeros(2, dtype=torch.float64, device=dev)
+    barrier = make_stream_barrier()
+    stream = torch.cuda.current_stream()
+
+    def one_step():
+        return zero2_step(shard, gptrs, params, wl.lr, stats, barrier)
+
+    for _ in range(args.warmup):
+        one_step()
+    t0 = shard.get_state()[2]
+    shard.reset_profile()
+    shard.set_profiling(True)
+    launches0 = shard.profile().launches
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            one_step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    dist.barrier()
+    assert shard.get_state()[2] - t0 == args.steps, "timed ZeRO-2 steps were skipped (overflow)"
+    prof = shard.profile()
+    shard.set_profiling(False)
+    ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
+    ms_step = ms / args.steps
+    p2_ms = prof.update_pass_ms / prof.steps
+    peak, peak_kind = hbm_peak()
+    nv_bytes = plan["nvlink_read_bytes"] + plan["nvlink_write_bytes"]
+    # pass 2 of a rank: reads the FP32 sum and master/m/v, writes master/m/v
+    # and the 16-bit cast to itself and to the (N - 1) peers
+    p2_bytes = (4 + 12 + 12 + 2 * ws) * n
+    if ws == 1:  # no peers: pass 2 against the HBM copy bandwidth
+        roofline = {"bound": "hbm", "kernel": "adam_kernel (pass 2, FP32 sum)", "avg_launch_ms": p2_ms,
+                    "alg_bytes_per_launch": p2_bytes, "achieved": p2_bytes / (p2_ms * 1e-3) / 1e9, "peak": peak,
+                    "unit": "GB/s", "frac": p2_bytes / (p2_ms * 1e-3) / 1e9 / peak, "peak_kind": peak_kind,
+                    "traffic": None}
+    else:  # the bytes each rank moves per direction over NVLink against the measured peer copy
+        per_dir = plan["nvlink_read_bytes"] / (ms_step * 1e-3) / 1e9
+        roofline = {"bound": "nvlink", "kernel": "whole step (pass 1 peer loads, pass 2 peer stores)",
+                    "alg_bytes_per_step_per_direction": plan["nvlink_read_bytes"], "achieved": per_dir,
+                    "peak": 770.0, "unit": "GB/s", "frac": per_dir / 770.0,
+                    "peak_kind": "measured peer copy per direction on this pool", "traffic": None,
+                    "pass2_avg_launch_ms": p2_ms}
+    line = {
+        "metric": METRIC + " (ZeRO-2 over peer memory)", "value": N * args.steps / (ms * 1e-3) / 1e9, "unit": UNIT,
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "impl": "b200",
+        "config": {"workload": wl.name, "numel_model": N, "numel_per_rank": n, "grad_buffers_per_step": ws,
+                   "weights": "bf16" if wl.bf16 else "fp16", "predivide": float(ws),
+                   "parallelism": f"zero2 over {ws} ranks: gradient reduce-scatter fused with pass 1 (peer loads), "
+                                  "weight all-gather fused with the cast (peer stores), 16-byte statistics "
+                                  "all-reduce, stream barriers before and after the step",
+                   "l2": "inputs far above the 126 MB L2; no flush"},
+        "nvlink": {"bytes_per_rank_per_step": nv_bytes, "read_bytes": plan["nvlink_read_bytes"],
+                   "write_bytes": plan["nvlink_write_bytes"],
+                   "achieved_gbs_per_rank_whole_step": nv_bytes / (ms_step * 1e-3) / 1e9 if nv_bytes else None,
+                   "reference_gbs_per_direction": 770.0},
+        "roofline": roofline,
+        "gpu_launches": prof.launches - launches0,
+        "clocks": clocks.summary(),
+    }
+    shard.close()
+    gmap.close()
+    wmap.close()
+    dist.barrier()
+    if own_group:
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -616,6 +845,8 @@ def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.zero2:
+        return run_zero2(args)
     if args.api == "multi":
         return run_multi(args)
     return run_b200(args)

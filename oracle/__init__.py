@@ -332,6 +332,36 @@ class OracleShard:
                        ctypes.byref(self.scaler), lr, ctypes.byref(info))
         return info
 
+    def step_threaded(self, grads, lr: float, threads: int, chunk: int = 1 << 22) -> StepInfo:
+        """The same step with the index range cut into contiguous chunks, run
+        on `threads` host threads: pass 1 chunk by chunk (the chunk sums added
+        in index order), the decision, then the update chunk by chunk.  Every
+        element's state is that of step(); only the double sum of squares is
+        re-associated at the chunk boundaries.  (For timing the oracle on all
+        host cores.)"""
+        grads = [np.ascontiguousarray(g, dtype=np.uint16) for g in grads]
+        n = self.master.size
+        assert all(g.size == n for g in grads)
+        inv_pre, inv_us = ingest_factors(len(grads), self.hp.predivide, self.scaler.scale)
+        bad, ssum = grad_stats(grads, self.gbf16, inv_pre, inv_us, threads=threads, chunk=chunk)
+        info = step_decide(self.hp, self.scaler, lr, bad, ssum)
+        if info.overflow or n == 0:
+            return info
+
+        def run(lo):
+            hi = min(n, lo + chunk)
+            sub = [g[lo:hi] for g in grads]
+            if self.hp.optimizer == 1:
+                sgd_apply(None, lo, sub, self.gbf16, self.segs, self.master[lo:hi], self.w[lo:hi], self.wbf16,
+                          self.hp, lr, info)
+            else:
+                adam_apply(None, lo, sub, self.gbf16, self.segs, self.master[lo:hi], self.m[lo:hi], self.v[lo:hi],
+                           self.w[lo:hi], self.wbf16, self.hp, lr, info)
+
+        with ThreadPoolExecutor(max(1, threads)) as ex:
+            list(ex.map(run, range(0, n, chunk)))
+        return info
+
 
 @dataclass
 class Oracle64Shard:

@@ -3,6 +3,8 @@ by, and the source hash that ties recorded ncu counters to the kernel code."""
 import os
 import shutil
 
+import pytest
+
 import bench
 
 
@@ -36,3 +38,30 @@ def test_source_hash_ignores_comments_but_not_code(tmp_path):
         assert bench.kernel_source_hash() != h0
     finally:
         bench.KERNEL_SRCS = orig
+
+
+def test_zero2_plan_tiles_the_model():
+    """Every rank's slice and segment table of the ZeRO-2 mode: equal slices
+    that tile the model, segment tables that tile each slice with the
+    model's weight decays, and the NVLink bytes of one step."""
+    import bench
+    from synth import workloads as W
+    wl = W.pythia_1p4b()
+    for world in (1, 2, 4, 8):
+        covered = []
+        for r in range(world):
+            p = bench.zero2_plan(wl, world, r)
+            assert p["n"] * world == wl.numel and p["lo"] == r * p["n"]
+            pos = 0
+            for off, cnt, wd in p["segments"]:
+                assert off == pos and cnt > 0
+                g = p["lo"] + off     # the model's segment containing this piece has the same decay
+                src = [s for s in wl.segments if s[0] <= g < s[0] + s[1]][0]
+                assert wd == src[2] and g + cnt <= src[0] + src[1]
+                pos += cnt
+            assert pos == p["n"]
+            assert p["nvlink_read_bytes"] == p["nvlink_write_bytes"] == (world - 1) * 2 * p["n"]
+            covered.append((p["lo"], p["n"]))
+        assert sum(c for _, c in covered) == wl.numel
+    with pytest.raises(ValueError):
+        bench.zero2_plan(W.tiny(), 3, 0)

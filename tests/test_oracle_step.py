@@ -485,3 +485,31 @@ def test_sgd_closed_form_and_untouched_moments(orc):
     np.testing.assert_allclose(sh.master, expect, rtol=2.0 ** -22, atol=lr * 2.0 ** -22)
     assert not sh.m.any() and not sh.v.any()
     np.testing.assert_array_equal(sh.w, f16(sh.master))
+
+
+@pytest.mark.parametrize("optimizer", [0, 1])
+def test_threaded_step_equals_single_threaded(orc, optimizer):
+    """The oracle split over host threads by contiguous chunks (the CPU
+    baseline on all cores) gives the single-threaded step's state byte for
+    byte, across segment and chunk boundaries and through an overflow; the
+    norm differs only by the re-association of the chunk sums."""
+    import synth
+    n = 100_003
+    segs = [(0, 40_000, 0.1), (40_000, 3, 0.0), (40_003, n - 40_003, 0.1)]
+    hp = orc.OracleHparams(clip_norm=1.0, init_scale=2.0 ** 12, scale_window=2, optimizer=optimizer)
+    master = synth.master_normal(n, 0.02, 5)
+    a = orc.OracleShard(master, hp, wbf16=True, gbf16=False, segments=segs)
+    b = orc.OracleShard(master, hp, wbf16=True, gbf16=False, segments=segs)
+    for s in range(1, 6):
+        g = synth.grad_normal16(n, 1e-3, a.scale, 5, 0, s)
+        if s == 3:
+            g[70_001] = 0x7C00
+        ia = a.step([g], 1e-3)
+        ib = b.step_threaded([g], 1e-3, threads=4, chunk=7_777)
+        assert (ia.overflow, ia.scale_next, ia.t) == (ib.overflow, ib.scale_next, ib.t)
+        assert ia.overflow == (1 if s == 3 else 0)
+        if not ia.overflow:
+            assert abs(ia.norm - ib.norm) <= 1e-12 * ia.norm
+            assert ia.coef == ib.coef   # on these inputs the re-association does not reach the FP32 coefficient
+    for x, y in ((a.master, b.master), (a.m, b.m), (a.v, b.v), (a.w, b.w)):
+        assert x.tobytes() == y.tobytes()
