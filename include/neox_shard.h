@@ -230,7 +230,10 @@ neox_status neox_shard_apply(neox_shard* h, const void* const* grads, int32_t nu
  *         n = 0 removes the copies.  Each destination receives numel elements.
  * The pointers must stay valid for every later step; the vector layout takes
  * them into account (a destination with another residue mod 16 bytes makes
- * the kernels use narrower vectors). */
+ * the kernels use narrower vectors).  A destination in another rank's memory
+ * is written without any ordering against that rank's own work: its reads of
+ * the buffer must wait for this rank's step, and this rank's step must wait
+ * for its earlier reads (the ordering rules of the ZeRO-2 section below). */
 neox_status neox_shard_set_weight_copies(neox_shard* h, void* const* dsts, int32_t n);
 
 /* ------------------------------------------------------------------------
@@ -252,6 +255,28 @@ neox_status neox_shard_set_weight_copies(neox_shard* h, void* const* dsts, int32
  * stays in local memory for pass 2.  The split step's 16-byte all-reduce
  * then gives every rank the same decision, and neox_shard_set_weight_copies
  * pointed at the peers' full-weight buffers performs the all-gather.
+ *
+ * Ordering between the ranks is the caller's.  The library orders work only
+ * on the stream it is given and cannot see the peers' streams, so on every
+ * rank's stream the caller must place:
+ *   1. before the rank's pass 1 of a step (neox_shard_step or
+ *      neox_shard_grad_stats): a point after which every rank's gradient
+ *      buffer of that step is complete, because pass 1 reads the peers'
+ *      buffers;
+ *   2. after the rank's pass 2 (neox_shard_step or neox_shard_apply), before
+ *      the rank writes its gradient buffer again (its next backward) or reads
+ *      its full-weight buffer (its next forward): a point after which every
+ *      rank's step has finished, because pass 1 -- and pass 2, which re-reads
+ *      the gradients when no FP32 sum is kept (K < 5 without
+ *      NEOX_SHARD_ACCUMULATE) -- reads this rank's gradient buffer, and every
+ *      rank's pass 2 stores into this rank's full-weight buffer.
+ * Both are barriers across the ranks' streams: a one-element all-reduce
+ * (e.g. NCCL) enqueued on the step's stream, or interprocess events
+ * (cudaIpcGetEventHandle / cudaIpcOpenEventHandle) that each rank records
+ * on its stream and the others wait on with cudaStreamWaitEvent, once they
+ * know the record has been issued (a wait refers to the last record issued
+ * before it).  The statistics all-reduce between the passes is not such a
+ * point for either.  The Python package's zero.zero2_step places both.
  *
  * The calls below wrap CUDA IPC (one node; handles are plain bytes that the
  * caller exchanges, e.g. with torch.distributed).  Errors: NEOX_ERR_CUDA
@@ -346,7 +371,12 @@ neox_status neox_shard_reset_profile(neox_shard* h);
  * caller owns and keeps alive.  Each tensor chooses its own vector width and
  * head peel from its own pointers.  A tensor may have numel 0 (its pointers
  * are then ignored).  The steps are then launched with only the learning
- * rate; both kernels walk a chunk table (up to 65,536 elements per chunk).
+ * rate.  The tensors that stream 8-element vectors (those whose arrays share
+ * a 16-byte residue) form one sequence of vectors: pass 1 deals it to the
+ * threads with a fixed assignment (so the norm is deterministic), the SGD
+ * pass takes it in chunks from a counter; the AdamW pass takes the vectors
+ * of all tensors as one sequence in chunks from a counter; tensors with
+ * narrower vectors are covered grid-stride one after another.
  * ------------------------------------------------------------------------ */
 typedef struct {
     uint64_t numel;
@@ -368,8 +398,8 @@ typedef struct {
 typedef struct neox_multi neox_multi;
 
 /* Validate every tensor (NEOX_ERR_INVALID_ARGUMENT before any CUDA call),
- * build the chunk table and copy it, the tensor table and the gradient
- * pointer table to the device. */
+ * choose each tensor's layout, and copy the tensor table, the sequence table
+ * and the gradient pointer table to the device. */
 neox_status neox_multi_create(const neox_tensor_set* set, const neox_hparams* hp, int device, neox_multi** out);
 /* One step, as neox_shard_step (blocking on cuda_stream). */
 neox_status neox_multi_step(neox_multi* h, float lr, void* cuda_stream, neox_step_result* out);
@@ -379,7 +409,7 @@ neox_status neox_multi_step_async(neox_multi* h, float lr, const float* lr_devic
 /* Point the tensors at other gradient buffers: `grads` is a host array of
  * ntensors * num_grads device pointers (tensor-major), each with the same
  * address residue as the buffer it replaces (the tensor's vector layout is
- * kept).  Waits for the device, then copies the table (synchronous). */
+ * kept).  Waits for the device, then copies the tables (synchronous). */
 neox_status neox_multi_rebind_grads(neox_multi* h, const void* const* grads);
 neox_status neox_multi_set_hparams(neox_multi* h, const neox_hparams* hp);
 neox_status neox_multi_get_state(const neox_multi* h, float* scale, int32_t* good, int64_t* t);
@@ -425,9 +455,16 @@ const char* neox_multi_last_error(const neox_multi* h);
  * calling thread's current CUDA device and on cuda_stream; returns after the
  * step has finished (it synchronises cuda_stream only).
  *
- * Set-up: the first call on each device looks up the address of the static
- * array on that device (cudaGetSymbolAddress); make that first call before any
- * stream capture begins.
+ * Set-up: the first call on each device (with that device current) does the
+ * set-up: it checks the device, looks up the address of the static array on
+ * that device (cudaGetSymbolAddress; host code cannot use the array's name as
+ * a device address) and loads every kernel instance the call can launch --
+ * CUDA loads kernels lazily, at their first launch, which takes device memory
+ * -- so that no later call, whatever its dtypes, K or update rule, takes any.
+ * Make that first call before any stream capture begins, and before the
+ * memory it must not touch is handed out.  Every call looks the address up
+ * again (that allocates nothing) and repeats the set-up when the device's
+ * context is not the one it was done in (after cudaDeviceReset, say).
  *
  * Sharing: every call on a device uses the same static array, and the array
  * keeps the previous call's contents.  Each call reloads what must start

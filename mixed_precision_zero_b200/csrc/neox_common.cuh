@@ -244,6 +244,49 @@ __device__ __forceinline__ void ingest_batch(const PT& gp, int K, unsigned long 
         for (int e = 0; e < VEC; e++) g[u][e] = __fmul_rn(g[u][e], inv_us);
 }
 
+// ingest_batch with the buffers taken two at a time: the 2U loads of buffers
+// k and k + 1 are issued before either is used (for K > 1 and a short U this
+// doubles the bytes each thread keeps in flight).  Per element the sum still
+// runs over the buffers in order, so the result is ingest_batch's.
+template <class G, int VEC, int U, class PT>
+__device__ __forceinline__ void ingest_batch_pairs(const PT& gp, int K, unsigned long long i0, unsigned long long di,
+                                                   float inv_pre, float inv_us, float (&g)[U][VEC]) {
+#pragma unroll
+    for (int u = 0; u < U; u++)
+#pragma unroll
+        for (int e = 0; e < VEC; e++) g[u][e] = 0.0f;
+    const bool pre1 = inv_pre == 1.0f;
+    int k = 0;
+    for (; k + 1 < K; k += 2) {
+        uint16_t h0[U][VEC], h1[U][VEC];
+#pragma unroll
+        for (int u = 0; u < U; u++) ld16<VEC>(gp[k] + i0 + u * di, h0[u]);
+#pragma unroll
+        for (int u = 0; u < U; u++) ld16<VEC>(gp[k + 1] + i0 + u * di, h1[u]);
+#pragma unroll
+        for (int u = 0; u < U; u++)
+#pragma unroll
+            for (int e = 0; e < VEC; e++) {
+                g[u][e] = __fadd_rn(g[u][e], pre1 ? G::dec(h0[u][e]) : __fmul_rn(G::dec(h0[u][e]), inv_pre));
+                g[u][e] = __fadd_rn(g[u][e], pre1 ? G::dec(h1[u][e]) : __fmul_rn(G::dec(h1[u][e]), inv_pre));
+            }
+    }
+    if (k < K) {
+        uint16_t h[U][VEC];
+#pragma unroll
+        for (int u = 0; u < U; u++) ld16<VEC>(gp[k] + i0 + u * di, h[u]);
+#pragma unroll
+        for (int u = 0; u < U; u++)
+#pragma unroll
+            for (int e = 0; e < VEC; e++)
+                g[u][e] = __fadd_rn(g[u][e], pre1 ? G::dec(h[u][e]) : __fmul_rn(G::dec(h[u][e]), inv_pre));
+    }
+#pragma unroll
+    for (int u = 0; u < U; u++)
+#pragma unroll
+        for (int e = 0; e < VEC; e++) g[u][e] = __fmul_rn(g[u][e], inv_us);
+}
+
 // ingest_batch for the last strides of a range: vector u is ingested only
 // when ok[u]; the loads of all valid vectors are still issued together.
 template <class G, int VEC, int U, class PT>

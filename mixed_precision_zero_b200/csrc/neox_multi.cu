@@ -13,15 +13,24 @@
 //
 // Work decomposition.  Each tensor keeps its own vector width and peeled
 // head, chosen from its own pointers; its head and ragged tail are done by
-// block (tensor index mod grid).
-//  * Pass 1 and the SGD pass walk the tensors in order and cover each one
-//    grid-stride across the whole grid, starting where the previous tensor
-//    left off (no synchronisation between tensors).
-//  * The AdamW pass treats the vectors of all tensors as one sequence and
-//    hands it out in chunks from the counter in the scalar block, as the flat
-//    pass does.
-// A static decomposition into per-block chunks (every block streaming its own
-// distant region) was measured 11% slower than the grid-stride.
+// block (tensor index mod grid).  The tensors whose arrays share a 16-byte
+// residue -- nearly always all of them -- stream 8-element vectors, and their
+// vectors form one sequence, tensor after tensor (the MtSeq table):
+//  * Pass 1 deals the sequence to the threads with a fixed assignment
+//    (thread g takes vectors g, g + S, g + 2S, ...; S = threads of the grid),
+//    four per batch, so the norm is deterministic and the batches run full
+//    across tensor ends.  On the Pythia-1.4B layout as 290 tensors the
+//    earlier per-tensor grid-stride, whose last batch of every tensor ran
+//    partly empty and which formed each tensor's starting thread with a
+//    64-bit modulo, took 0.59 ms against 0.44 for the flat pass.
+//  * The SGD pass takes the sequence in chunks of four-vector batches from
+//    the counter in the scalar block, as the flat SGD pass does.
+//  * The AdamW pass takes the vectors of all tensors (any width) as one
+//    sequence in chunks from the same counter, as the flat AdamW pass does.
+// Tensors with narrower vectors are covered grid-stride, tensor by tensor,
+// after the sequence.  A static decomposition into per-block chunks (every
+// block streaming its own distant region) was measured 11% slower than the
+// grid-stride.
 
 #include "neox_shard.h"
 #include "neox_common.cuh"
@@ -36,8 +45,6 @@ namespace {
 
 constexpr int kMtThreads1 = 512;
 constexpr int kMtThreads3 = 256;
-constexpr int kMtDescBatch = 256;  // pass 1: tensor descriptors staged in shared memory at a time
-constexpr int kMtDescBatch3 = 768; // pass 2 (SGD): 60 KB of descriptors (dynamic shared memory)
 constexpr int kMtChunk = 2;        // pass 2 (AdamW): vectors per thread in each chunk taken from the counter
 
 struct alignas(16) MtTensor {
@@ -69,20 +76,157 @@ __device__ __forceinline__ unsigned long long rotated_start(unsigned long long b
     return g >= r ? g - r : g + n - r;
 }
 
-// Copy descriptors [base, base + cnt) into shared memory (all threads).  A
-// warp then reads each tensor's pointers from shared memory instead of
-// waiting on a dependent global load at every tensor boundary.
-__device__ __forceinline__ void stage_descriptors(const MtTensor* __restrict__ tens, int base, int cnt,
-                                                  MtTensor* tsh) {
-    constexpr int W = sizeof(MtTensor) / 16;
-    const int4* src = reinterpret_cast<const int4*>(tens + base);
-    int4* dst = reinterpret_cast<int4*>(tsh);
-    __syncthreads();  // the previous batch is no longer read
-    for (int i = threadIdx.x; i < cnt * W; i += blockDim.x) dst[i] = __ldg(src + i);
-    __syncthreads();
+// ---------------------------------------------------------------- pass 1
+// The 8-element vectors of all tensors whose layout has VEC = 8 (every tensor
+// whose arrays share a 16-byte residue, i.e. nearly always) form one
+// sequence, tensor after tensor.  Entry t of this table describes the t-th
+// such tensor: sequence vector gv (end_{t-1} <= gv < end_t) is its elements
+// off0 + 8 gv ... off0 + 8 gv + 7.
+struct alignas(16) MtSeq {
+    unsigned long long end;  // one past the tensor's last vector in the sequence
+    long long off0;          // element index of sequence vector gv: off0 + 8 * gv
+    const uint16_t* g0;      // the tensor's first gradient buffer
+    int gbase;               // its K gradient pointers are gtab[gbase .. gbase + K)
+    float wd;                // its weight decay
+    float* master;           // (the SGD pass) its FP32 master weights
+    uint16_t* w;             //                its 16-bit working weights
+};
+static_assert(sizeof(MtSeq) == 48, "three 16-byte words; pass 1 reads the first two");
+
+// A thread's position in the sequence table.  Its vectors come in increasing
+// order, so the cursor only moves forward; over the whole pass a thread
+// crosses each tensor boundary at most once.
+struct SeqCursor {
+    int t = -1;
+    unsigned long long end = 0;
+    long long off0 = 0;
+    const uint16_t* g0 = nullptr;
+    int gbase = 0;
+    __device__ __forceinline__ void to(const MtSeq* __restrict__ seq, unsigned long long gv) {
+        while (gv >= end) {
+            ++t;
+            const int4 a = __ldg(reinterpret_cast<const int4*>(seq + t));
+            const int4 b = __ldg(reinterpret_cast<const int4*>(seq + t) + 1);
+            end = (unsigned long long)(unsigned)a.x | ((unsigned long long)(unsigned)a.y << 32);
+            off0 = (long long)((unsigned long long)(unsigned)a.z | ((unsigned long long)(unsigned)a.w << 32));
+            g0 = reinterpret_cast<const uint16_t*>((unsigned long long)(unsigned)b.x |
+                                                   ((unsigned long long)(unsigned)b.y << 32));
+            gbase = b.z;
+        }
+    }
+};
+
+// U vectors whose gradient addresses are known, ingested together: for every
+// buffer the U loads are issued before any is used.  ok[u] = false leaves
+// vector u zero (no load).  Per element the arithmetic is ingest()'s.
+template <class G, int U, bool PRED>
+__device__ __forceinline__ void seq_ingest(const uint16_t* const (&a0)[U], const long long (&el)[U],
+                                           const int (&gb)[U], const bool (&ok)[U],
+                                           const uint16_t* const* __restrict__ gtab, int K, float inv_pre,
+                                           float inv_us, float (&g)[U][8]) {
+    const bool pre1 = inv_pre == 1.0f;  // x * 1 == x exactly: skip the multiply
+#pragma unroll
+    for (int u = 0; u < U; u++)
+#pragma unroll
+        for (int e = 0; e < 8; e++) g[u][e] = 0.0f;
+    for (int k = 0; k < K; k++) {
+        uint16_t h[U][8];
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+            if (!PRED || ok[u]) {
+                ld16<8>(k == 0 ? a0[u] : gtab[gb[u] + k] + el[u], h[u]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; e++) h[u][e] = 0;
+            }
+        }
+        if (pre1) {
+#pragma unroll
+            for (int u = 0; u < U; u++)
+#pragma unroll
+                for (int e = 0; e < 8; e++) g[u][e] = __fadd_rn(g[u][e], G::dec(h[u][e]));
+        } else {
+#pragma unroll
+            for (int u = 0; u < U; u++)
+#pragma unroll
+                for (int e = 0; e < 8; e++) g[u][e] = __fadd_rn(g[u][e], __fmul_rn(G::dec(h[u][e]), inv_pre));
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < U; u++)
+#pragma unroll
+        for (int e = 0; e < 8; e++) g[u][e] = __fmul_rn(g[u][e], inv_us);
 }
 
-// ---------------------------------------------------------------- pass 1
+// Pass 1 over the sequence, with a fixed assignment of vectors to threads:
+// thread g takes sequence vectors g, g + S, g + 2S, ... (S = threads of the
+// grid), U of them per batch whose loads are issued together, and sums its
+// squares in that order, so the norm is deterministic.  The batches run full
+// across tensor ends (a per-tensor grid-stride leaves the last batch of every
+// tensor partly empty).  A batch whose U vectors lie in one tensor -- nearly
+// every batch, the vectors being S apart -- addresses them from one base as
+// the flat pass does; a batch across a tensor end moves the cursor vector by
+// vector; the last, partial batch is predicated.
+template <class G, int KFIX>
+__device__ __forceinline__ void mt_p1_seq(const MtSeq* __restrict__ seq, unsigned long long total,
+                                          const uint16_t* const* __restrict__ gtab, int K_rt, float inv_pre,
+                                          float inv_us, double& s, int& bad) {
+    const int K = KFIX ? KFIX : K_rt;
+    constexpr int U = KFIX ? 4 : 2;
+    const unsigned long long S = (unsigned long long)gridDim.x * kMtThreads1;
+    SeqCursor cur;
+    unsigned long long v = (unsigned long long)blockIdx.x * kMtThreads1 + threadIdx.x;
+    for (; v + (U - 1) * S < total; v += U * S) {
+        cur.to(seq, v);
+        const uint16_t* a0[U];
+        long long el[U];
+        int gb[U];
+        const bool ok[U] = {};
+        float g[U][8];
+        if (v + (U - 1) * S < cur.end) {  // one tensor: one base, constant strides
+#pragma unroll
+            for (int u = 0; u < U; u++) {
+                el[u] = cur.off0 + 8ll * (long long)v + 8ll * (long long)(u * S);
+                a0[u] = cur.g0 + el[u];
+                gb[u] = cur.gbase;
+            }
+        } else {
+#pragma unroll
+            for (int u = 0; u < U; u++) {
+                cur.to(seq, v + u * S);
+                el[u] = cur.off0 + 8ll * (long long)(v + u * S);
+                a0[u] = cur.g0 + el[u];
+                gb[u] = cur.gbase;
+            }
+        }
+        seq_ingest<G, U, false>(a0, el, gb, ok, gtab, K, inv_pre, inv_us, g);
+#pragma unroll
+        for (int u = 0; u < U; u++) s += vec_sumsq<8>(g[u], bad);
+    }
+    if (v < total) {  // the last, partial batch
+        const uint16_t* a0[U];
+        long long el[U];
+        int gb[U];
+        bool ok[U];
+        float g[U][8];
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+            ok[u] = v + u * S < total;
+            if (ok[u]) cur.to(seq, v + u * S);
+            el[u] = cur.off0 + 8ll * (long long)(v + u * S);
+            a0[u] = cur.g0 + el[u];
+            gb[u] = cur.gbase;
+        }
+        seq_ingest<G, U, true>(a0, el, gb, ok, gtab, K, inv_pre, inv_us, g);
+#pragma unroll
+        for (int u = 0; u < U; u++)
+            if (ok[u]) s += vec_sumsq<8>(g[u], bad);
+    }
+}
+
+// Pass 1 over one tensor with narrower vectors (arrays without a common
+// 16-byte residue), grid-stride across the whole grid from the tensor's
+// rotated start, U strides per batch.
 template <class G, int VEC, int KFIX>
 __device__ __forceinline__ void mt_p1_tensor(const GradTab& gp, int K_rt, const MtTensor& T, float inv_pre,
                                              float inv_us, double& s, int& bad) {
@@ -96,9 +240,6 @@ __device__ __forceinline__ void mt_p1_tensor(const GradTab& gp, int K_rt, const 
 #pragma unroll
         for (int u = 0; u < U; u++) s += vec_sumsq<VEC>(g[u], bad);
     }
-    // The last (fewer than U) strides: still U loads in flight.  Most tensors
-    // of a model are shorter than U grid strides, so this batch does most of
-    // their work.  The thread's vectors are summed in the same order.
     if (v < T.nvec) {
         bool ok[U];
 #pragma unroll
@@ -115,52 +256,57 @@ template <class G, int KFIX>
 __device__ __forceinline__ void mt_p1_dispatch(const MtTensor& T, const GradTab& gp, int K, float inv_pre,
                                                float inv_us, double& s, int& bad) {
     switch (T.vec) {
-        case 8: mt_p1_tensor<G, 8, KFIX>(gp, K, T, inv_pre, inv_us, s, bad); break;
         case 4: mt_p1_tensor<G, 4, KFIX>(gp, K, T, inv_pre, inv_us, s, bad); break;
         case 2: mt_p1_tensor<G, 2, KFIX>(gp, K, T, inv_pre, inv_us, s, bad); break;
         default: mt_p1_tensor<G, 1, KFIX>(gp, K, T, inv_pre, inv_us, s, bad); break;
     }
 }
 
+// Pass 1: the sequence of 8-element vectors, then the tensors with narrower
+// vectors (`odd`, normally none), then every tensor's peeled head and ragged
+// tail (tensor t by block t mod grid), each thread summing in that fixed
+// order; then the shared end of pass 1 (finish_pass1).
 template <class G>
 __global__ void __launch_bounds__(kMtThreads1, 1024 / kMtThreads1)
-mt_stats_kernel(const MtTensor* __restrict__ tens, int ntensors, const uint16_t* const* __restrict__ gtab, int K,
-                ScalerArgs sa, double* __restrict__ part_s, int* __restrict__ part_b, DevScalars* __restrict__ sc) {
+mt_stats_kernel(const MtTensor* __restrict__ tens, int ntensors, const MtSeq* __restrict__ seq,
+                unsigned long long total8, const int* __restrict__ odd, int nodd,
+                const uint16_t* const* __restrict__ gtab, int K, ScalerArgs sa, double* __restrict__ part_s,
+                int* __restrict__ part_b, DevScalars* __restrict__ sc) {
     __shared__ double sh_s[kMtThreads1 / 32];
     __shared__ int sh_b[kMtThreads1 / 32];
     __shared__ bool is_last;
-    __shared__ MtTensor tsh[kMtDescBatch];
     const float inv_us = unscale_factor(sa.post, sc->scale);
     double s = 0.0;
     int bad = 0;
-    for (int base = 0; base < ntensors; base += kMtDescBatch) {
-    const int cnt = ntensors - base < kMtDescBatch ? ntensors - base : kMtDescBatch;
-    stage_descriptors(tens, base, cnt, tsh);
-    for (int ti = base; ti < base + cnt; ti++) {
-        const MtTensor T = tsh[ti - base];  // by value: registers, not re-read after stores
-        if (T.numel == 0) continue;
+    if (K == 1) mt_p1_seq<G, 1>(seq, total8, gtab, K, sa.inv_pre, inv_us, s, bad);
+    else mt_p1_seq<G, 0>(seq, total8, gtab, K, sa.inv_pre, inv_us, s, bad);
+    for (int j = 0; j < nodd; j++) {
+        const MtTensor T = tens[__ldg(odd + j)];
         const GradTab gp{gtab, T.gbase};
         if (K == 1) mt_p1_dispatch<G, 1>(T, gp, K, sa.inv_pre, inv_us, s, bad);
         else mt_p1_dispatch<G, 0>(T, gp, K, sa.inv_pre, inv_us, s, bad);
-        if ((unsigned)ti % gridDim.x == blockIdx.x) {  // this tensor's head and tail
-            const unsigned long long tail0 = T.head + T.nvec * T.vec;
-            const unsigned long long extra = T.head + (T.numel - tail0);
-            for (unsigned long long j = threadIdx.x; j < extra; j += kMtThreads1) {
-                const unsigned long long i = j < T.head ? j : tail0 + (j - T.head);
-                float g[1];
-                ingest<G, 1>(gp, K, i, sa.inv_pre, inv_us, g);
-                s += vec_sumsq<1>(g, bad);
-            }
-        }
     }
+    for (int ti = blockIdx.x; ti < ntensors; ti += gridDim.x) {  // heads and ragged tails
+        const MtTensor T = tens[ti];
+        if (T.numel == 0) continue;
+        const GradTab gp{gtab, T.gbase};
+        const unsigned long long tail0 = T.head + T.nvec * T.vec;
+        const unsigned long long extra = T.head + (T.numel - tail0);
+        for (unsigned long long j = threadIdx.x; j < extra; j += kMtThreads1) {
+            const unsigned long long i = j < T.head ? j : tail0 + (j - T.head);
+            float g[1];
+            ingest<G, 1>(gp, K, i, sa.inv_pre, inv_us, g);
+            s += vec_sumsq<1>(g, bad);
+        }
     }
     finish_pass1<kMtThreads1>(s, bad, part_s, part_b, sc, sa, sh_s, sh_b, &is_last);
 }
 
 // ---------------------------------------------------------------- pass 2
-// Pass 2 with plain SGD over one tensor, grid-stride from the tensor's
-// rotated start, kUnrollSgd strides in flight per thread (its loads are too
-// few per vector to cover the memory latency one at a time).
+// Pass 2 with plain SGD over one tensor with narrower vectors, grid-stride
+// from the tensor's rotated start, kUnrollSgd strides in flight per thread
+// (its loads are too few per vector to cover the memory latency one at a
+// time).
 template <class G, class W, int VEC, int KFIX>
 __device__ __forceinline__ void mt_sgd_tensor(const GradTab& gp, int K_rt, const MtTensor& T, float keep1, float c,
                                               float inv_us, const AdamArgs& a) {
@@ -202,19 +348,107 @@ template <class G, class W, int KFIX>
 __device__ __forceinline__ void mt_sgd_dispatch(const MtTensor& T, const GradTab& gp, int K, float keep1, float c,
                                                 float inv_us, const AdamArgs& a) {
     switch (T.vec) {
-        case 8: mt_sgd_tensor<G, W, 8, KFIX>(gp, K, T, keep1, c, inv_us, a); break;
         case 4: mt_sgd_tensor<G, W, 4, KFIX>(gp, K, T, keep1, c, inv_us, a); break;
         case 2: mt_sgd_tensor<G, W, 2, KFIX>(gp, K, T, keep1, c, inv_us, a); break;
         default: mt_sgd_tensor<G, W, 1, KFIX>(gp, K, T, keep1, c, inv_us, a); break;
     }
 }
 
-// Pass 2 with plain SGD over every tensor, tensor by tensor (the AdamW pass
-// is mt_adam_chunked_kernel below).
+// The sequence cursor of the SGD pass: pass 1's, plus the tensor's master
+// and working-weight arrays and its decay factor fl32(1 - fl32(lr * wd)).
+struct SeqCursor2 {
+    int t = -1;
+    unsigned long long end = 0;
+    long long off0 = 0;
+    const uint16_t* g0 = nullptr;
+    int gbase = 0;
+    float keep = 1.0f;
+    float* master = nullptr;
+    uint16_t* w = nullptr;
+    __device__ __forceinline__ void to(const MtSeq* __restrict__ seq, unsigned long long gv, float lr) {
+        while (gv >= end) {
+            ++t;
+            const int4* q = reinterpret_cast<const int4*>(seq + t);
+            const int4 a = __ldg(q), b = __ldg(q + 1), d = __ldg(q + 2);
+            end = (unsigned long long)(unsigned)a.x | ((unsigned long long)(unsigned)a.y << 32);
+            off0 = (long long)((unsigned long long)(unsigned)a.z | ((unsigned long long)(unsigned)a.w << 32));
+            g0 = reinterpret_cast<const uint16_t*>((unsigned long long)(unsigned)b.x |
+                                                   ((unsigned long long)(unsigned)b.y << 32));
+            gbase = b.z;
+            keep = __fsub_rn(1.0f, __fmul_rn(lr, __int_as_float(b.w)));
+            master = reinterpret_cast<float*>((unsigned long long)(unsigned)d.x | ((unsigned long long)(unsigned)d.y << 32));
+            w = reinterpret_cast<uint16_t*>((unsigned long long)(unsigned)d.z | ((unsigned long long)(unsigned)d.w << 32));
+        }
+    }
+};
+
+// Pass 2 with plain SGD: the sequence of 8-element vectors in chunks of
+// kUnrollSgd x kMtThreads3 vectors taken from the counter in the scalar block
+// (zeroed by pass 1's last block, which this grid waits for) -- the flat SGD
+// pass's scheme.  A thread's kUnrollSgd vectors of a chunk are loaded as one
+// batch when they lie in one tensor, as they do in nearly every chunk; a
+// chunk that crosses a tensor end goes one vector at a time.  The cursor only
+// moves forward: a block's chunks, and a thread's vectors in a chunk, come in
+// increasing order.
 template <class G, class W>
-__device__ __forceinline__ void mt_sgd_update(const MtTensor* __restrict__ tens, int ntensors,
-                                          const uint16_t* const* __restrict__ gtab, int K, const AdamArgs& a_arg,
-                                          const DevScalars* __restrict__ sc) {
+__device__ __forceinline__ void mt_sgd_seq(const MtSeq* __restrict__ seq, unsigned long long total,
+                                           const uint16_t* const* __restrict__ gtab, int K, float c, float inv_us,
+                                           const AdamArgs& a, DevScalars* __restrict__ sc) {
+    constexpr int U = kUnrollSgd;
+    constexpr unsigned long long kChunk = (unsigned long long)kMtThreads3 * U;
+    constexpr unsigned long long kDi = (unsigned long long)kMtThreads3 * 8;  // elements between a thread's vectors
+    const unsigned long long nchunks = (total + kChunk - 1) / kChunk;
+    __shared__ unsigned int chunk_sh;
+    SeqCursor2 cur;
+    for (;;) {
+        if (threadIdx.x == 0) chunk_sh = atomicAdd(&sc->chunk_next, 1u);
+        __syncthreads();
+        const unsigned long long ch = chunk_sh;
+        __syncthreads();                  // chunk_sh is rewritten by the next iteration
+        if (ch >= nchunks) break;         // uniform across the block
+        const unsigned long long gv0 = ch * kChunk + threadIdx.x;
+        if (gv0 >= total) continue;
+        cur.to(seq, gv0, a.lr);
+        if (gv0 + (U - 1) * kMtThreads3 < cur.end) {  // the thread's U vectors lie in one tensor
+            const unsigned long long el0 = (unsigned long long)(cur.off0 + 8ll * (long long)gv0);
+            const GradTab gp{gtab, cur.gbase};
+            float g[U][8], p[U][8], keep[8];
+            ingest_batch<G, 8, U>(gp, K, el0, kDi, a.inv_pre, inv_us, g);
+#pragma unroll
+            for (int u = 0; u < U; u++) ld32<8>(cur.master + el0 + u * kDi, p[u]);
+#pragma unroll
+            for (int e = 0; e < 8; e++) keep[e] = cur.keep;
+#pragma unroll
+            for (int u = 0; u < U; u++) {
+                sgd_vec<8>(g[u], keep, c, a.lr, p[u]);
+                st32<8>(cur.master + el0 + u * kDi, p[u]);
+                st16<W, 8>(cur.w + el0 + u * kDi, p[u]);
+            }
+        } else {
+            for (int u = 0; u < U; u++) {
+                const unsigned long long gv = gv0 + (unsigned long long)u * kMtThreads3;
+                if (gv >= total) break;
+                cur.to(seq, gv, a.lr);
+                const unsigned long long el = (unsigned long long)(cur.off0 + 8ll * (long long)gv);
+                const GradTab gp{gtab, cur.gbase};
+                float g[8], p[8], keep[8];
+                ingest<G, 8>(gp, K, el, a.inv_pre, inv_us, g);
+                ld32<8>(cur.master + el, p);
+#pragma unroll
+                for (int e = 0; e < 8; e++) keep[e] = cur.keep;
+                sgd_vec<8>(g, keep, c, a.lr, p);
+                st32<8>(cur.master + el, p);
+                st16<W, 8>(cur.w + el, p);
+            }
+        }
+    }
+}
+
+template <class G, class W>
+__global__ void __launch_bounds__(kMtThreads3, 2)
+mt_sgd_kernel(const MtTensor* __restrict__ tens, int ntensors, const MtSeq* __restrict__ seq,
+              unsigned long long total8, const int* __restrict__ odd, int nodd,
+              const uint16_t* const* __restrict__ gtab, int K, AdamArgs a_arg, DevScalars* __restrict__ sc) {
     asm volatile("griddepcontrol.wait;" ::: "memory");  // pass 1's results
     if (sc->overflow) return;
     const float c = sc->coef;
@@ -225,33 +459,29 @@ __device__ __forceinline__ void mt_sgd_update(const MtTensor* __restrict__ tens,
         a.step_size = sc->step_size;
         a.bcs = sc->bc2_sqrt;
     }
-    // Descriptors are staged in dynamic shared memory, kMtDescBatch3 at a time,
-    // so that a warp reads each tensor's pointers from shared memory instead of
-    // waiting on a dependent global load at every tensor boundary.
-    extern __shared__ MtTensor tsh_dyn[];
-    for (int base = 0; base < ntensors; base += kMtDescBatch3) {
-    const int cnt = ntensors - base < kMtDescBatch3 ? ntensors - base : kMtDescBatch3;
-    stage_descriptors(tens, base, cnt, tsh_dyn);
-    for (int ti = base; ti < base + cnt; ti++) {
-        const MtTensor T = tsh_dyn[ti - base];  // by value: registers, not re-read after stores
-        if (T.numel == 0) continue;
+    mt_sgd_seq<G, W>(seq, total8, gtab, K, c, inv_us, a, sc);
+    for (int j = 0; j < nodd; j++) {
+        const MtTensor T = tens[__ldg(odd + j)];
         const GradTab gp{gtab, T.gbase};
         const float keep1 = __fsub_rn(1.0f, __fmul_rn(a.lr, T.wd));  // fl32(1 - fl32(lr * wd))
         if (K == 1) mt_sgd_dispatch<G, W, 1>(T, gp, K, keep1, c, inv_us, a);
         else mt_sgd_dispatch<G, W, 0>(T, gp, K, keep1, c, inv_us, a);
-        if ((unsigned)ti % gridDim.x == blockIdx.x) {  // this tensor's head and tail
-            const unsigned long long tail0 = T.head + T.nvec * T.vec;
-            const unsigned long long extra = T.head + (T.numel - tail0);
-            for (unsigned long long j = threadIdx.x; j < extra; j += kMtThreads3) {
-                const unsigned long long i = j < T.head ? j : tail0 + (j - T.head);
-                float g[1], p[1] = {T.master[i]}, keep[1] = {keep1};
-                ingest<G, 1>(gp, K, i, a.inv_pre, inv_us, g);
-                sgd_vec<1>(g, keep, c, a.lr, p);
-                T.master[i] = p[0];
-                T.w[i] = W::enc(p[0]);
-            }
-        }
     }
+    for (int ti = blockIdx.x; ti < ntensors; ti += gridDim.x) {  // heads and ragged tails
+        const MtTensor T = tens[ti];
+        if (T.numel == 0) continue;
+        const GradTab gp{gtab, T.gbase};
+        const float keep1 = __fsub_rn(1.0f, __fmul_rn(a.lr, T.wd));
+        const unsigned long long tail0 = T.head + T.nvec * T.vec;
+        const unsigned long long extra = T.head + (T.numel - tail0);
+        for (unsigned long long j = threadIdx.x; j < extra; j += kMtThreads3) {
+            const unsigned long long i = j < T.head ? j : tail0 + (j - T.head);
+            float g[1], p[1] = {T.master[i]}, keep[1] = {keep1};
+            ingest<G, 1>(gp, K, i, a.inv_pre, inv_us, g);
+            sgd_vec<1>(g, keep, c, a.lr, p);
+            T.master[i] = p[0];
+            T.w[i] = W::enc(p[0]);
+        }
     }
 }
 
@@ -359,14 +589,8 @@ mt_adam_chunked_kernel(const MtTensor* __restrict__ tens, int ntensors, const ui
     }
 }
 
-template <class G, class W>
-__global__ void __launch_bounds__(kMtThreads3)
-mt_sgd_kernel(const MtTensor* __restrict__ tens, int ntensors, const uint16_t* const* __restrict__ gtab, int K,
-              AdamArgs a, const DevScalars* __restrict__ sc) {
-    mt_sgd_update<G, W>(tens, ntensors, gtab, K, a, sc);
-}
-
-using MtSgdKernel = void (*)(const MtTensor*, int, const uint16_t* const*, int, AdamArgs, const DevScalars*);
+using MtSgdKernel = void (*)(const MtTensor*, int, const MtSeq*, unsigned long long, const int*, int,
+                             const uint16_t* const*, int, AdamArgs, DevScalars*);
 using MtAdamKernel = void (*)(const MtTensor*, int, const uint16_t* const*, int, AdamArgs, DevScalars*,
                               unsigned long long);
 
@@ -402,6 +626,11 @@ struct neox_multi {
     int max_parts = 0;
     MtTensor* d_tens = nullptr;
     const uint16_t** d_gtab = nullptr;
+    MtSeq* d_seq = nullptr;             // pass 1: the sequence of 8-element vectors
+    int* d_odd = nullptr;               // pass 1: tensors with narrower vectors
+    int nseq = 0, nodd = 0;
+    unsigned long long total8 = 0;      // vectors in the sequence
+    std::vector<int> seq_tensor;        // tensor index of each sequence entry
     DevScalars* d_sc = nullptr;
     double* d_part_s = nullptr;
     int* d_part_b = nullptr;
@@ -431,6 +660,8 @@ neox_status mcuda_fail(neox_multi* h, cudaError_t e, const char* what) {
 void mfree(neox_multi* h) {
     if (h->d_tens) cudaFree(h->d_tens);
     if (h->d_gtab) cudaFree(h->d_gtab);
+    if (h->d_seq) cudaFree(h->d_seq);
+    if (h->d_odd) cudaFree(h->d_odd);
     if (h->d_sc) cudaFree(h->d_sc);
     if (h->d_part_s) cudaFree(h->d_part_s);
     if (h->d_part_b) cudaFree(h->d_part_b);
@@ -480,6 +711,36 @@ std::string build_tables(const neox_tensor_set* set, std::vector<MtTensor>& tens
     return "";
 }
 
+// Pass 1's sequence table (tensors with VEC = 8, in order) and the list of
+// the other non-empty tensors, from the tensor table and the gradient table.
+void build_sequence(const std::vector<MtTensor>& tens, const std::vector<const uint16_t*>& gtab, int K,
+                    std::vector<MtSeq>& seq, std::vector<int>& seq_tensor, std::vector<int>& odd,
+                    unsigned long long& total8) {
+    seq.clear();
+    seq_tensor.clear();
+    odd.clear();
+    total8 = 0;
+    for (int ti = 0; ti < (int)tens.size(); ti++) {
+        const MtTensor& T = tens[ti];
+        if (T.numel == 0 || T.nvec == 0) continue;
+        if (T.vec != 8) {
+            odd.push_back(ti);
+            continue;
+        }
+        MtSeq e{};
+        e.off0 = (long long)T.head - 8ll * (long long)total8;
+        total8 += T.nvec;
+        e.end = total8;
+        e.g0 = gtab[(size_t)ti * K];
+        e.gbase = ti * K;
+        e.wd = T.wd;
+        e.master = T.master;
+        e.w = T.w;
+        seq.push_back(e);
+        seq_tensor.push_back(ti);
+    }
+}
+
 // Resident-grid size for the multi-tensor kernels (at most one vector of all
 // the tensors' vectors per thread).
 template <class Kern>
@@ -507,8 +768,8 @@ neox_status mt_enqueue(neox_multi* h, float lr, const float* lr_dev, cudaStream_
     {
         auto k1 = h->gdtype == NEOX_FP16 ? mt_stats_kernel<F16> : mt_stats_kernel<BF16>;
         const int grid = h->grid1;
-        k1<<<grid, kMtThreads1, 0, st>>>(h->d_tens, h->ntensors, h->d_gtab, h->K, sa, h->d_part_s, h->d_part_b,
-                                         h->d_sc);
+        k1<<<grid, kMtThreads1, 0, st>>>(h->d_tens, h->ntensors, h->d_seq, h->total8, h->d_odd, h->nodd, h->d_gtab,
+                                         h->K, sa, h->d_part_s, h->d_part_b, h->d_sc);
         if ((e = cudaGetLastError()) != cudaSuccess) return mcuda_fail(h, e, "pass-1 launch");
         h->prof.launches += 1;
     }
@@ -518,7 +779,7 @@ neox_status mt_enqueue(neox_multi* h, float lr, const float* lr_dev, cudaStream_
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(sgd ? h->grid2_sgd : h->grid2);
         cfg.blockDim = dim3(kMtThreads3);
-        cfg.dynamicSmemBytes = sgd ? sizeof(MtTensor) * kMtDescBatch3 : 0;
+        cfg.dynamicSmemBytes = 0;
         cfg.stream = st;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -528,8 +789,12 @@ neox_status mt_enqueue(neox_multi* h, float lr, const float* lr_dev, cudaStream_
         const MtTensor* tens = h->d_tens;
         const uint16_t* const* gtab = h->d_gtab;
         if (sgd) {
-            const DevScalars* sc = h->d_sc;
-            e = cudaLaunchKernelEx(&cfg, mt_sgd_kernel_for(h->gdtype, h->wdtype), tens, h->ntensors, gtab, h->K, a, sc);
+            DevScalars* sc = h->d_sc;
+            const MtSeq* seq = h->d_seq;
+            const int* odd = h->d_odd;
+            const unsigned long long total8 = h->total8;
+            e = cudaLaunchKernelEx(&cfg, mt_sgd_kernel_for(h->gdtype, h->wdtype), tens, h->ntensors, seq, total8, odd,
+                                   h->nodd, gtab, h->K, a, sc);
         } else {
             DevScalars* sc = h->d_sc;
             const unsigned long long total = h->total_vecs;
@@ -626,16 +891,13 @@ neox_status neox_multi_create(const neox_tensor_set* set, const neox_hparams* hp
             st = mcuda_fail(nullptr, e, "cudaMemcpy scalars");
             goto done;
         }
-        // The SGD pass runs with kMtDescBatch3 descriptors of dynamic shared
-        // memory; the AdamW pass reads descriptors as its chunks reach them.
-        // Both grids are set here (set_hparams may switch the rule).
+        // Both update passes' grids are set here (set_hparams may switch the
+        // rule).  The SGD pass takes its work in chunks of the sequence.
         const MtAdamKernel k2 = mt_adam_kernel_for(h->gdtype, h->wdtype);
         const MtSgdKernel k2s = mt_sgd_kernel_for(h->gdtype, h->wdtype);
-        const int dyn = (int)(sizeof(MtTensor) * kMtDescBatch3);
         int occ = 0, occ_sgd = 0;
-        if ((e = cudaFuncSetAttribute(k2s, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn)) != cudaSuccess ||
-            (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k2, kMtThreads3, 0)) != cudaSuccess ||
-            (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_sgd, k2s, kMtThreads3, dyn)) != cudaSuccess) {
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k2, kMtThreads3, 0)) != cudaSuccess ||
+            (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_sgd, k2s, kMtThreads3, 0)) != cudaSuccess) {
             st = mcuda_fail(nullptr, e, "configuring the update kernel");
             goto done;
         }
@@ -654,6 +916,20 @@ neox_status neox_multi_create(const neox_tensor_set* set, const neox_hparams* hp
             before += T.nvec;
         }
         h->tens = tens;
+        std::vector<MtSeq> seq;
+        std::vector<int> odd;
+        build_sequence(tens, gtab, h->K, seq, h->seq_tensor, odd, h->total8);
+        h->nseq = (int)seq.size();
+        h->nodd = (int)odd.size();
+        if ((e = cudaMalloc(&h->d_seq, sizeof(MtSeq) * (seq.empty() ? 1 : seq.size()))) != cudaSuccess ||
+            (e = cudaMalloc(&h->d_odd, sizeof(int) * (odd.empty() ? 1 : odd.size()))) != cudaSuccess ||
+            (!seq.empty() && (e = cudaMemcpy(h->d_seq, seq.data(), sizeof(MtSeq) * seq.size(),
+                                             cudaMemcpyHostToDevice)) != cudaSuccess) ||
+            (!odd.empty() && (e = cudaMemcpy(h->d_odd, odd.data(), sizeof(int) * odd.size(),
+                                             cudaMemcpyHostToDevice)) != cudaSuccess)) {
+            st = mcuda_fail(nullptr, e, "copying the sequence table");
+            goto done;
+        }
         if ((!tens.empty() && (e = cudaMemcpy(h->d_tens, tens.data(), sizeof(MtTensor) * tens.size(),
                                               cudaMemcpyHostToDevice)) != cudaSuccess) ||
             (!gtab.empty() && (e = cudaMemcpy(h->d_gtab, gtab.data(), sizeof(void*) * gtab.size(),
@@ -704,10 +980,16 @@ neox_status neox_multi_rebind_grads(neox_multi* h, const void* const* grads) {
             gtab[(size_t)ti * h->K + k] = static_cast<const uint16_t*>(p);
         }
     }
+    std::vector<MtSeq> seq;
+    std::vector<int> seq_tensor, odd;
+    unsigned long long total8 = 0;
+    build_sequence(h->tens, gtab, h->K, seq, seq_tensor, odd, total8);  // same layout: only g0 changes
     DeviceGuard g(h->device);
     cudaError_t e = cudaDeviceSynchronize();
     if (e == cudaSuccess && !gtab.empty())
         e = cudaMemcpy(h->d_gtab, gtab.data(), sizeof(void*) * gtab.size(), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && !seq.empty())
+        e = cudaMemcpy(h->d_seq, seq.data(), sizeof(MtSeq) * seq.size(), cudaMemcpyHostToDevice);
     if (e != cudaSuccess) return mcuda_fail(h, e, "updating the gradient table");
     return NEOX_OK;
 }

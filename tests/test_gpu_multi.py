@@ -20,16 +20,22 @@ WDS = [0.1, 0.0, 0.1, 0.05, 0.0, 0.1, 0.1, 0.0, 0.1, 0.1]
 
 
 class MultiCase:
-    def __init__(self, K=1, hp=None, wbf16=False, gbf16=False, seed=3, lr=6e-4):
+    def __init__(self, K=1, hp=None, wbf16=False, gbf16=False, seed=3, lr=6e-4, same_offset=False):
+        """same_offset: every array of tensor i starts at the same element
+        offset, so every tensor streams 8-element vectors (pass 1 takes them
+        as one sequence) after a peeled head; otherwise the arrays of most
+        tensors have different residues and narrower vectors."""
         self.K, self.lr, self.seed, self.gbf16 = K, lr, seed, gbf16
         self.hp = hp or Hparams()
         wdt = torch.bfloat16 if wbf16 else torch.float16
         gdt = torch.bfloat16 if gbf16 else torch.float16
         self.parts = []
         for i, (n, off, wd) in enumerate(zip(SIZES, OFFSETS, WDS)):
+            woff = off if same_offset else (off * 3) % 8
+            goff = [off if same_offset else (off + k) % 8 for k in range(K)]
             p = {"n": n, "wd": wd, "master": Guarded(n, torch.float32, off), "m": Guarded(n, torch.float32, off),
-                 "v": Guarded(n, torch.float32, off), "w": Guarded(n, wdt, (off * 3) % 8),
-                 "g": [Guarded(n, gdt, (off + k) % 8) for k in range(K)]}
+                 "v": Guarded(n, torch.float32, off), "w": Guarded(n, wdt, woff),
+                 "g": [Guarded(n, gdt, goff[k]) for k in range(K)]}
             if n:
                 synth.gpu_master_normal(p["master"].t, 0.02, seed, tensor_id=i)
                 p["m"].t.zero_()
@@ -105,6 +111,23 @@ def test_multi_with_clip_and_overflow(K, pre):
         res, info = c.step()
         assert res.overflow == (1 if s == 3 else 0)
         c.check(res, info)
+    c.shard.close()
+
+
+@pytest.mark.parametrize("K,bf16", [(1, False), (3, True)])
+def test_multi_sequence_path_bit_exact(K, bf16):
+    """Every tensor on 8-element vectors after its head (pass 1 deals all of
+    them to the threads as one sequence), K buffers each: bit-exact against
+    the oracle with clipping off, through an overflow in the last buffer."""
+    c = MultiCase(K=K, hp=Hparams(clip_norm=0.0, predivide=float(K), init_scale=2.0 ** 12, scale_window=2),
+                  wbf16=bf16, gbf16=bf16, lr=1e-3, same_offset=True)
+    for s in range(1, 6):
+        c.gen(s, 3e-3)
+        if s == 2:
+            c.parts[8]["g"][K - 1].t.view(torch.int16)[12345] = 0x7F80 if bf16 else 0x7C00
+        res, info = c.step()
+        assert res.overflow == (1 if s == 2 else 0)
+        c.check(res, info, exact=True)
     c.shard.close()
 
 
