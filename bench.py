@@ -572,7 +572,11 @@ def run_b200(args):
     # are double-buffered, so the copy for step s + 1 (on a copy stream)
     # overlaps step s (neox_shard_step_async, whose result the GPU writes into
     # pinned host memory).  Several ranks: the split step, one after the other.
-    host_grads = [g.cpu().pin_memory() for g in grads]
+    host_grads = []
+    for g in grads:  # straight into pinned memory: one host copy per buffer, not two
+        hg = torch.empty(g.shape, dtype=g.dtype, pin_memory=True)
+        hg.copy_(g)
+        host_grads.append(hg)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if ws > 1:

@@ -382,6 +382,8 @@ struct SeqCursor2 {
     }
 };
 
+// (The AdamW pass's split tiles measured 425 against 458 Gparams/s in this
+// pass, and are not used here.)
 // Pass 2 with plain SGD: the sequence of 8-element vectors in chunks of
 // kUnrollSgd x kMtThreads3 vectors taken from the counter in the scalar block
 // (zeroed by pass 1's last block, which this grid waits for) -- the flat SGD
@@ -506,6 +508,38 @@ __device__ __forceinline__ void mt_adam_one(const GradTab& gp, int K_rt, const M
     st16<W, VEC>(T.w + i, p);
 }
 
+// One AdamW vector of a split tile: elements i0 + [0, 4) and i0 + 128 + [0, 4)
+// of tensor T (lane t of a tile whose 32 vectors lie in T takes i0 = the
+// tile's first element + 4t), so that each warp-wide FP32 access covers 512
+// contiguous bytes.
+template <class G, class W, int KFIX>
+__device__ __forceinline__ void mt_adam_split(const GradTab& gp, int K_rt, const MtTensor& T, unsigned long long i0,
+                                              float keep1, float c, float inv_us, const AdamArgs& a) {
+    const int K = KFIX ? KFIX : K_rt;
+    const unsigned long long i1 = i0 + 128;
+    float g0[4], g1[4], p0[4], p1[4], m0[4], m1[4], v0[4], v1[4], keep[4];
+#pragma unroll
+    for (int e = 0; e < 4; e++) keep[e] = keep1;
+    ingest<G, 4>(gp, K, i0, a.inv_pre, inv_us, g0);
+    ingest<G, 4>(gp, K, i1, a.inv_pre, inv_us, g1);
+    ld32<4>(T.master + i0, p0);
+    ld32<4>(T.master + i1, p1);
+    ld32<4>(T.m + i0, m0);
+    ld32<4>(T.m + i1, m1);
+    ld32<4>(T.v + i0, v0);
+    ld32<4>(T.v + i1, v1);
+    adam_vec<4>(g0, keep, c, a, p0, m0, v0);
+    adam_vec<4>(g1, keep, c, a, p1, m1, v1);
+    st32<4>(T.master + i0, p0);
+    st32<4>(T.master + i1, p1);
+    st32<4>(T.m + i0, m0);
+    st32<4>(T.m + i1, m1);
+    st32<4>(T.v + i0, v0);
+    st32<4>(T.v + i1, v1);
+    st16<W, 4>(T.w + i0, p0);
+    st16<W, 4>(T.w + i1, p1);
+}
+
 template <class G, class W, int KFIX>
 __device__ __forceinline__ void mt_adam_one_dispatch(const GradTab& gp, int K, const MtTensor& T,
                                                      unsigned long long vi, float keep1, float c, float inv_us,
@@ -565,8 +599,18 @@ mt_adam_chunked_kernel(const MtTensor* __restrict__ tens, int ntensors, const ui
                 keep1 = __fsub_rn(1.0f, __fmul_rn(a.lr, T.wd));  // fl32(1 - fl32(lr * wd))
             }
             const GradTab gp{gtab, T.gbase};
-            if (K == 1) mt_adam_one_dispatch<G, W, 1>(gp, K, T, gv - T.before, keep1, c, inv_us, a);
-            else mt_adam_one_dispatch<G, W, 0>(gp, K, T, gv - T.before, keep1, c, inv_us, a);
+            const unsigned int lane = threadIdx.x & 31;
+            const unsigned long long tile = gv - lane;  // the warp's 32 consecutive vectors
+            if (T.vec == 8 && tile >= T.before && tile + 31 < tend) {
+                // the tile lies in T (so every lane of the warp sees it): split it
+                const unsigned long long i0 = T.head + 8 * (tile - T.before) + 4ull * lane;
+                if (K == 1) mt_adam_split<G, W, 1>(gp, K, T, i0, keep1, c, inv_us, a);
+                else mt_adam_split<G, W, 0>(gp, K, T, i0, keep1, c, inv_us, a);
+            } else if (K == 1) {
+                mt_adam_one_dispatch<G, W, 1>(gp, K, T, gv - T.before, keep1, c, inv_us, a);
+            } else {
+                mt_adam_one_dispatch<G, W, 0>(gp, K, T, gv - T.before, keep1, c, inv_us, a);
+            }
         }
     }
     for (int ti = blockIdx.x; ti < ntensors; ti += gridDim.x) {  // heads and tails
