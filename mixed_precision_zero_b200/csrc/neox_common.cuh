@@ -287,6 +287,39 @@ __device__ __forceinline__ void ingest_batch_pairs(const PT& gp, int K, unsigned
         for (int e = 0; e < VEC; e++) g[u][e] = __fmul_rn(g[u][e], inv_us);
 }
 
+// U split vectors: vector u is the 4 elements at i0 + u*di and the 4 at
+// i0 + u*di + 128 (g[u][0..3] and g[u][4..7]).  All 2U loads of a buffer are
+// issued before any is used.  Per element the arithmetic is ingest()'s, over
+// the buffers in order.
+template <class G, int U, class PT>
+__device__ __forceinline__ void ingest_halves(const PT& gp, int K, unsigned long long i0, unsigned long long di,
+                                              float inv_pre, float inv_us, float (&g)[U][8]) {
+#pragma unroll
+    for (int u = 0; u < U; u++)
+#pragma unroll
+        for (int e = 0; e < 8; e++) g[u][e] = 0.0f;
+    const bool pre1 = inv_pre == 1.0f;
+    for (int k = 0; k < K; k++) {
+        uint16_t a[U][4], b[U][4];
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+            ld16<4>(gp[k] + i0 + u * di, a[u]);
+            ld16<4>(gp[k] + i0 + u * di + 128, b[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < U; u++)
+#pragma unroll
+            for (int e = 0; e < 4; e++) {
+                g[u][e] = __fadd_rn(g[u][e], pre1 ? G::dec(a[u][e]) : __fmul_rn(G::dec(a[u][e]), inv_pre));
+                g[u][4 + e] = __fadd_rn(g[u][4 + e], pre1 ? G::dec(b[u][e]) : __fmul_rn(G::dec(b[u][e]), inv_pre));
+            }
+    }
+#pragma unroll
+    for (int u = 0; u < U; u++)
+#pragma unroll
+        for (int e = 0; e < 8; e++) g[u][e] = __fmul_rn(g[u][e], inv_us);
+}
+
 // ingest_batch for the last strides of a range: vector u is ingested only
 // when ok[u]; the loads of all valid vectors are still issued together.
 template <class G, int VEC, int U, class PT>

@@ -358,6 +358,7 @@ __device__ __forceinline__ void mt_sgd_dispatch(const MtTensor& T, const GradTab
 // and working-weight arrays and its decay factor fl32(1 - fl32(lr * wd)).
 struct SeqCursor2 {
     int t = -1;
+    unsigned long long start = 0;  // the tensor's first vector in the sequence
     unsigned long long end = 0;
     long long off0 = 0;
     const uint16_t* g0 = nullptr;
@@ -370,6 +371,7 @@ struct SeqCursor2 {
             ++t;
             const int4* q = reinterpret_cast<const int4*>(seq + t);
             const int4 a = __ldg(q), b = __ldg(q + 1), d = __ldg(q + 2);
+            start = end;
             end = (unsigned long long)(unsigned)a.x | ((unsigned long long)(unsigned)a.y << 32);
             off0 = (long long)((unsigned long long)(unsigned)a.z | ((unsigned long long)(unsigned)a.w << 32));
             g0 = reinterpret_cast<const uint16_t*>((unsigned long long)(unsigned)b.x |
@@ -382,14 +384,13 @@ struct SeqCursor2 {
     }
 };
 
-// (The AdamW pass's split tiles measured 425 against 458 Gparams/s in this
-// pass, and are not used here.)
 // Pass 2 with plain SGD: the sequence of 8-element vectors in chunks of
 // kUnrollSgd x kMtThreads3 vectors taken from the counter in the scalar block
 // (zeroed by pass 1's last block, which this grid waits for) -- the flat SGD
-// pass's scheme.  A thread's kUnrollSgd vectors of a chunk are loaded as one
-// batch when they lie in one tensor, as they do in nearly every chunk; a
-// chunk that crosses a tensor end goes one vector at a time.  The cursor only
+// pass's scheme.  When a warp's kUnrollSgd tiles lie in one tensor, as in
+// nearly every chunk, they take the split tiles of the flat passes, loaded as
+// one batch; otherwise a thread's vectors are loaded as one batch when they
+// lie in one tensor, and one at a time across a tensor end.  The cursor only
 // moves forward: a block's chunks, and a thread's vectors in a chunk, come in
 // increasing order.
 template <class G, class W>
@@ -411,7 +412,45 @@ __device__ __forceinline__ void mt_sgd_seq(const MtSeq* __restrict__ seq, unsign
         const unsigned long long gv0 = ch * kChunk + threadIdx.x;
         if (gv0 >= total) continue;
         cur.to(seq, gv0, a.lr);
-        if (gv0 + (U - 1) * kMtThreads3 < cur.end) {  // the thread's U vectors lie in one tensor
+        const unsigned int lane = threadIdx.x & 31;
+        const unsigned long long tile = gv0 - lane;  // the warp's 32 consecutive vectors start here
+        if (tile >= cur.start && tile + (U - 1) * kMtThreads3 + 31 < cur.end) {
+            // the warp's U tiles lie in one tensor (then every lane of the warp
+            // sees it): split them as the flat passes do, lane t taking elements
+            // 4t + [0, 4) and 128 + 4t + [0, 4) of each tile, all 2U gradient
+            // halves loaded as one batch
+            const unsigned long long b0 = (unsigned long long)(cur.off0 + 8ll * (long long)tile) + 4ull * lane;
+            const GradTab gp{gtab, cur.gbase};
+            float g[U][8], p[U][8], keep[8];
+            ingest_halves<G, U>(gp, K, b0, kDi, a.inv_pre, inv_us, g);
+#pragma unroll
+            for (int u = 0; u < U; u++) {
+                float lo[4], hi[4];
+                ld32<4>(cur.master + b0 + u * kDi, lo);
+                ld32<4>(cur.master + b0 + u * kDi + 128, hi);
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                    p[u][e] = lo[e];
+                    p[u][4 + e] = hi[e];
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < 8; e++) keep[e] = cur.keep;
+#pragma unroll
+            for (int u = 0; u < U; u++) {
+                sgd_vec<8>(g[u], keep, c, a.lr, p[u]);
+                float lo[4], hi[4];
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                    lo[e] = p[u][e];
+                    hi[e] = p[u][4 + e];
+                }
+                st32<4>(cur.master + b0 + u * kDi, lo);
+                st32<4>(cur.master + b0 + u * kDi + 128, hi);
+                st16<W, 4>(cur.w + b0 + u * kDi, lo);
+                st16<W, 4>(cur.w + b0 + u * kDi + 128, hi);
+            }
+        } else if (gv0 + (U - 1) * kMtThreads3 < cur.end) {  // the thread's U vectors lie in one tensor
             const unsigned long long el0 = (unsigned long long)(cur.off0 + 8ll * (long long)gv0);
             const GradTab gp{gtab, cur.gbase};
             float g[U][8], p[U][8], keep[8];

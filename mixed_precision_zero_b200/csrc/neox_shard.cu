@@ -172,10 +172,10 @@ __device__ __forceinline__ void keep_at(SegCursor& cur, unsigned long long i, co
 //  SGD: chunks of kUnrollSgd x kThreads3 vectors from the same counter, each
 //    thread's kUnrollSgd vectors loaded as one batch (its loads are too few
 //    per vector to cover the memory latency one at a time): 6.55 TB/s,
-//    against 6.27 for the static grid-stride with the same batches.  It
-//    keeps eight consecutive elements per lane: the AdamW pass's split tiles,
-//    with the two halves' loads issued as two batches, measured 425 against
-//    461 Gparams/s here.
+//    against 6.27 for the static grid-stride with the same batches.  Chunks
+//    of whole tiles use the AdamW pass's split tiles, all 2U gradient halves
+//    loaded as one batch: 6.66 against 6.57 TB/s (468 against 462 Gparams/s
+//    for the step); loading the two halves as two batches measured 425.
 template <bool SGD, class G, class W, int VEC, bool READ_ACC, int KFIX, bool COPIES, bool CHUNKED>
 __device__ __forceinline__ void pass2_vectors(const GradPtrs& gp, int K_rt, const float* __restrict__ acc,
                                               const Layout& L, const AdamArgs& a, float c, float inv_us,
@@ -199,6 +199,57 @@ __device__ __forceinline__ void pass2_vectors(const GradPtrs& gp, int K_rt, cons
             const unsigned long long ch = chunk_sh;
             __syncthreads();                  // chunk_sh is rewritten by the next iteration
             if (ch >= nchunks) break;         // uniform across the block
+            if constexpr (VEC == 8 && !READ_ACC) {
+                if ((ch + 1) * kChunk <= (L.nvec & ~31ull)) {
+                    // the whole chunk in split tiles, the AdamW pass's mapping: lane t
+                    // of warp j takes elements 4t + [0, 4) and 128 + 4t + [0, 4) of
+                    // tile 32 ch + 8u + j, u = 0..U-1; the 2U gradient halves are
+                    // loaded as one batch, then the 2U master halves
+                    constexpr unsigned long long kDi = (unsigned long long)kThreads3 * 8;
+                    const unsigned long long b0 = L.head + ch * kChunk * 8 + (threadIdx.x >> 5) * 256 +
+                                                  (threadIdx.x & 31) * 4;
+                    float g[U][8], p[U][8];
+                    ingest_halves<G, U>(gp, K, b0, kDi, a.inv_pre, inv_us, g);
+#pragma unroll
+                    for (int u = 0; u < U; u++) {
+                        float lo[4], hi[4];
+                        ld32<4>(master + b0 + u * kDi, lo);
+                        ld32<4>(master + b0 + u * kDi + 128, hi);
+#pragma unroll
+                        for (int e = 0; e < 4; e++) {
+                            p[u][e] = lo[e];
+                            p[u][4 + e] = hi[e];
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < U; u++) {
+                        const unsigned long long i0 = b0 + u * kDi, i1 = i0 + 128;
+                        float keep[8], lo[4], hi[4], klo[4], khi[4];
+                        keep_at<4>(cur, i0, seg_end, seg_wd, nsegs, a.lr, klo);
+                        keep_at<4>(cur, i1, seg_end, seg_wd, nsegs, a.lr, khi);
+#pragma unroll
+                        for (int e = 0; e < 4; e++) {
+                            keep[e] = klo[e];
+                            keep[4 + e] = khi[e];
+                        }
+                        sgd_vec<8>(g[u], keep, c, a.lr, p[u]);
+#pragma unroll
+                        for (int e = 0; e < 4; e++) {
+                            lo[e] = p[u][e];
+                            hi[e] = p[u][4 + e];
+                        }
+                        st32<4>(master + i0, lo);
+                        st32<4>(master + i1, hi);
+                        st16<W, 4>(w + i0, lo);
+                        st16<W, 4>(w + i1, hi);
+                        if constexpr (COPIES) {
+                            store_copies<W, 4>(wc, i0, lo);
+                            store_copies<W, 4>(wc, i1, hi);
+                        }
+                    }
+                    continue;
+                }
+            }
             const unsigned long long v0 = ch * kChunk + threadIdx.x;
             bool ok[U];
 #pragma unroll

@@ -69,7 +69,7 @@ class ShardCase:
 
     def __init__(self, n, *, K=1, wbf16=False, gbf16=False, hp: Hparams | None = None, lr=6e-4,
                  segments=None, default_wd=0.1, max_grads=1, offsets=None, seed=0, master_sigma=0.02,
-                 seg_init=None):
+                 seg_init=None, accumulate=False):
         self.n, self.K, self.lr = n, K, lr
         self.wbf16, self.gbf16 = wbf16, gbf16
         self.hp = hp or Hparams()
@@ -94,7 +94,8 @@ class ShardCase:
         self.segments = segments
         self.shard = NeoxShard(self.master.t, self.m.t, self.v.t, self.hp,
                                wdtype=_torch_dtype(wbf16), gdtype=_torch_dtype(gbf16),
-                               segments=segments, weight_decay=default_wd, max_grads=max_grads)
+                               segments=segments, weight_decay=default_wd, max_grads=max_grads,
+                               accumulate=accumulate)
         ohp = oracle_hparams(self.hp)
         master_host = self.master.t.cpu().numpy()
         self.orc = oracle.OracleShard(master_host, ohp, wbf16=wbf16, gbf16=gbf16, segments=segments,

@@ -119,6 +119,26 @@ def test_multi_buffer_predivide(K, max_grads, pre):
     c.close()
 
 
+@pytest.mark.parametrize("K,off,bf16", [(1, 0, False), (1, 3, True), (3, 5, False)])
+def test_accumulate_flag_bit_exact(K, off, bf16):
+    """NEOX_SHARD_ACCUMULATE at any K: pass 1 writes the FP32 sum (in split
+    tiles), pass 2 reads it.  Clip off: bit-exact with the oracle, through an
+    overflow, on a shard with whole tiles, a partial tile and a peeled head."""
+    n = 3_000_013
+    hp = Hparams(clip_norm=0.0, predivide=float(K), init_scale=2.0 ** 12, scale_window=2)
+    c = ShardCase(n, K=K, hp=hp, wbf16=bf16, gbf16=bf16, offsets={"all": off}, accumulate=True, lr=1e-3)
+    for s in range(1, 6):
+        c.gen_normal(s, 2e-3)
+        if s == 3:
+            c.inject(s, buffer=K - 1)
+        res, info = c.step()
+        c.check_result(res, info)
+        assert res.overflow == (1 if s == 3 else 0)
+        c.check_state(exact=True)
+    assert c.guards_intact()
+    c.close()
+
+
 def test_pythia_shaped_segments_small():
     """A 2-layer, hidden-64 model with the Pythia layout: 26 segments, wd 0 on
     biases and LayerNorms, LayerNorm weights initialised to one."""
