@@ -102,8 +102,9 @@ class IpcEventBarrier:
     has issued its waits of round r (that needs the host barrier of round
     r + 1), so no wait ever takes a later round's record for its own.
 
-    `event`, `open_event` and `host_barrier` are injectable for tests of the
-    protocol without a GPU."""
+    `event`, `open_event`, `host_barrier` and `exchange` (the all-gather of
+    the event handles) are injectable for tests of the protocol without a
+    GPU."""
 
     def __init__(self, group=None, *, event=None, open_event=None, host_barrier=None, exchange=None):
         import torch.distributed as dist
