@@ -275,14 +275,27 @@ def sample_inputs_host(wl, n_sample, threads, rank_seed=0):
     return lo, master, grads
 
 
+def oracle_sample_size(wl) -> int:
+    """Elements of the threaded oracle baseline: the whole workload when its
+    host copy (FP32 master/m/v, 16-bit weights and K gradient buffers) takes
+    less than half the host's available memory, else a 2^27-element slice."""
+    need = wl.numel * (18 + 2 * wl.K)   # the input master, the oracle's master/m/v/w, the gradients
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except Exception:
+        avail = 0
+    return wl.numel if need < avail // 2 else min(wl.numel, 1 << 27)
+
+
 def sample_inputs_device(wl, n_sample, master_dev, grads_dev):
     """The same kind of sample copied from the workload resident on the GPU
     (its bytes come from the CUDA twin of the generator): (lo, master, grads)."""
     import numpy as np
     import torch
     lo, n = cpu_sample_range(wl, n_sample)
-    master = master_dev[lo:lo + n].cpu().numpy().copy()
-    grads = [g[lo:lo + n].view(torch.int16).cpu().numpy().view(np.uint16).copy() for g in grads_dev]
+    master = master_dev[lo:lo + n].cpu().numpy()
+    grads = [g[lo:lo + n].view(torch.int16).cpu().numpy().view(np.uint16) for g in grads_dev]
     return lo, master, grads
 
 
@@ -291,11 +304,13 @@ def run_oracle_sample(wl, inputs, steps, seconds, threads=1, optimizer="adamw"):
     passed) over a contiguous sample of the workload, single-threaded or split
     over `threads` host threads by contiguous ranges.  The inputs are drawn
     before, untimed."""
+    import numpy as np
+
     import oracle
     lo, master, grads = inputs
     n = master.size
     segs, inits = sample_segments(wl, lo, n)
-    master = master.astype("float32", copy=True)
+    master = np.asarray(master, dtype=np.float32)   # the caller's sample: initialised in place
     for init, a, c in inits:
         if init == "zero":
             master[a:a + c] = 0
@@ -632,12 +647,15 @@ def run_b200(args):
         # slices of the resident workload (the bytes the GPU stepped on)
         cores = host_cores()
         master_dev = state[0]
-        out = run_oracle_sample(wl, sample_inputs_device(wl, 1 << 27, master_dev, grads), 50,
+        n_thr = oracle_sample_size(wl)
+        out = run_oracle_sample(wl, sample_inputs_device(wl, n_thr, master_dev, grads), 50,
                                 args.cpu_seconds, threads=cores, optimizer=args.optimizer)
         sec = sum(out["times"])
+        what = (f"the whole {wl.name} shard ({out['n']} elements)" if out["n"] == wl.numel else
+                f"{out['n']} contiguous elements of {wl.name} (from index {out['lo']})")
         cpu = {"value": out["n"] * len(out["times"]) / sec / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle",
-               "sample": f"{len(out['times'])} steps over {out['n']} contiguous elements of {wl.name} "
-                         f"(from index {out['lo']}), split over {cores} host threads by contiguous ranges"}
+               "sample": f"{len(out['times'])} steps over {what}, split over {cores} host threads by "
+                         "contiguous ranges"}
         out = run_oracle_sample(wl, sample_inputs_device(wl, 1 << 24, master_dev, grads), 50,
                                 args.cpu_seconds / 3, threads=1, optimizer=args.optimizer)
         sec = sum(out["times"])
