@@ -65,3 +65,20 @@ def test_zero2_plan_tiles_the_model():
         assert sum(c for _, c in covered) == wl.numel
     with pytest.raises(ValueError):
         bench.zero2_plan(W.tiny(), 3, 0)
+
+
+def test_parallel_generation_equals_one_call():
+    """The reference arm draws its inputs in contiguous chunks on several
+    threads; the counter-based generator makes that the same array as one
+    call, chunk boundaries (not multiples of 4) included."""
+    import numpy as np
+
+    import synth
+    n, lo = 50_021, 7
+    one = synth.grad_normal16(n, 1e-3, 2.0 ** 12, 3, 1, 2, True, start=lo)
+    par = bench.parallel_gen(synth.grad_normal16, n, 4, chunk=4_099, sigma=1e-3, scale=2.0 ** 12, seed=3,
+                             tensor_id=1, step=2, bf16=True, start=lo)
+    assert np.array_equal(one, par)
+    m1 = synth.master_normal(n, 0.02, 5, start=lo)
+    m2 = bench.parallel_gen(synth.master_normal, n, 3, chunk=10_001, sigma=0.02, seed=5, tensor_id=0, start=lo)
+    assert np.array_equal(m1, m2)
