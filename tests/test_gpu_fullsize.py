@@ -333,3 +333,46 @@ def test_accum8_30_call_trace():
     flags, scale, t = _trace_property(W.accum8_predivide(), 30)
     assert flags[0] == 1 and 0 in flags
     assert flags[19] == 1 and flags[24] == 1  # rate injections on calls 20 and 25
+
+
+def test_multi_tensor_full_size_equals_flat():
+    """The 1.41e9-parameter Pythia-shaped shard as 290 separately addressed
+    tensors (the multi-tensor entry point, as `bench.py --api multi` runs it)
+    against the flat step on a copy of the same bytes, which the exact-mode
+    tests tie to the oracle.  Clip off, so both sides apply coefficient 1:
+    every byte of master, m, v and the 16-bit copy must agree after every
+    call, through an overflow on call 2."""
+    from mixed_precision_zero_b200 import NeoxMultiShard
+    wl = W.pythia_1p4b()
+    n = wl.numel
+    hp = Hparams(wl.beta1, wl.beta2, wl.eps, 0.0, wl.predivide, wl.init_scale, 2.0, 1.0, wl.scale_window)
+    master = torch.empty(n, dtype=torch.float32, device="cuda")
+    synth.gpu_master_normal(master, wl.master_sigma, wl.seed)
+    for so, sc, _, init in wl.segments:
+        if init == "zero":
+            master[so:so + sc].zero_()
+        elif init == "one":
+            master[so:so + sc].fill_(1.0)
+    a = [master, torch.zeros_like(master), torch.zeros_like(master), master.to(torch.float16)]
+    b = [x.clone() for x in a]
+    g = torch.empty(n, dtype=torch.float16, device="cuda")
+    segs = wl.seg_table()
+    flat = NeoxShard(a[0], a[1], a[2], hp, segments=segs)
+    multi = NeoxMultiShard([{"master": b[0][o:o + c], "exp_avg": b[1][o:o + c], "exp_avg_sq": b[2][o:o + c],
+                             "params": b[3][o:o + c], "grads": [g[o:o + c]], "weight_decay": w}
+                            for o, c, w in segs], hp)
+    for s in range(1, 4):
+        synth.gpu_grad_normal16(g, wl.grad_sigma, flat.get_state()[0], wl.seed, 0, s)
+        if s == 2:
+            g.view(torch.int16)[synth.inject_index(n, wl.seed, s)] = 0x7C00
+        ra = flat.step([g], a[3], wl.lr)
+        rb = multi.step(wl.lr)
+        assert (ra.overflow, ra.loss_scale_next, ra.applied_steps) == (rb.overflow, rb.loss_scale_next, rb.applied_steps)
+        assert ra.overflow == (1 if s == 2 else 0)
+        if not ra.overflow:
+            assert abs(ra.grad_norm - rb.grad_norm) <= 1e-6 * ra.grad_norm
+        for x, y in zip(a, b):
+            assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))
+    flat.close()
+    multi.close()
+    del a, b, g, master
