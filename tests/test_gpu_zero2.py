@@ -1,4 +1,4 @@
-"""ZeRO-2 through peer memory, as two processes sharing one GPU.
+"""ZeRO-2 through peer memory, as two or three processes sharing one GPU.
 
 Each process is a data-parallel rank that owns one flat slice of the model
 and holds the full gradient of its own micro-batches and a full copy of the
@@ -100,10 +100,9 @@ def _rank_main(rank, world, port, q, cfg):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("accumulate,clip", [(True, 0.0), (False, 1.0)])
-def test_zero2_reduce_scatter_and_allgather_through_ipc(accumulate, clip):
+@pytest.mark.parametrize("world,accumulate,clip", [(2, True, 0.0), (2, False, 1.0), (3, True, 0.0), (3, False, 0.0)])
+def test_zero2_reduce_scatter_and_allgather_through_ipc(world, accumulate, clip):
     import torch.multiprocessing as mp
-    world = 2
     cfg = {"n": 300_007, "steps": 5, "lr": 1e-3, "overflow_step": 3, "accumulate": accumulate,
            "hp": {"clip_norm": clip, "init_scale": 2.0 ** 12, "scale_window": 2, "predivide": 2.0}}
     ctx = mp.get_context("spawn")

@@ -1,4 +1,4 @@
-"""The ZeRO-2 step's cross-rank ordering, on CPU (gloo, 2 ranks).
+"""The ZeRO-2 step's cross-rank ordering, on CPU (gloo, 2 and 3 ranks).
 
 zero.IpcEventBarrier orders the ranks' streams with interprocess CUDA events:
 record this rank's event of the round's parity, a host barrier (only to know
@@ -78,8 +78,8 @@ def _rank_barrier(rank, world, port, counts, q):
         dist.destroy_process_group()
 
 
-def test_ipc_event_barrier_waits_refer_to_the_same_round():
-    world = 2
+@pytest.mark.parametrize("world", [2, 3])
+def test_ipc_event_barrier_waits_refer_to_the_same_round(world):
     ctx = mp.get_context("spawn")
     mgr = ctx.Manager()
     counts = mgr.dict()
@@ -93,10 +93,9 @@ def test_ipc_event_barrier_waits_refer_to_the_same_round():
         p.join(timeout=60)
         assert p.exitcode == 0
     for rank, r, waits in got:
-        peer = 1 - rank
-        # one wait per round, on the peer's event of this round's parity, and it
-        # refers to the peer's (r // 2 + 1)-th record of that event: this round's
-        assert waits == [((peer, r % 2), r // 2 + 1)], (rank, r, waits)
+        # one wait per other rank and round, on that rank's event of this round's
+        # parity, referring to its (r // 2 + 1)-th record of that event: this round's
+        assert waits == [((p, r % 2), r // 2 + 1) for p in range(world) if p != rank], (rank, r, waits)
 
 
 class _Shard:
