@@ -58,8 +58,9 @@ def sample_indices(n, segments=None):
 
 
 class FullRun:
-    def __init__(self, wl: W.Workload, seed_offset=0):
+    def __init__(self, wl: W.Workload, seed_offset=0, optimizer="adamw"):
         self.wl = wl
+        self.optimizer = optimizer
         n = wl.numel
         dt = torch.bfloat16 if wl.bf16 else torch.float16
         off = wl.elem_offset
@@ -78,11 +79,12 @@ class FullRun:
         self.m.t.zero_()
         self.v.t.zero_()
         self.w.t.copy_(self.master.t.to(dt))
-        self.hp = Hparams(wl.beta1, wl.beta2, wl.eps, wl.clip, wl.predivide, wl.init_scale, 2.0, 1.0, wl.scale_window)
+        self.hp = Hparams(wl.beta1, wl.beta2, wl.eps, wl.clip, wl.predivide, wl.init_scale, 2.0, 1.0, wl.scale_window,
+                          optimizer=optimizer)
         self.shard = NeoxShard(self.master.t, self.m.t, self.v.t, self.hp, wdtype=dt, gdtype=dt,
                                segments=wl.seg_table(), weight_decay=wl.weight_decay, max_grads=wl.K)
         self.ohp = oracle.OracleHparams(wl.beta1, wl.beta2, wl.eps, wl.clip, wl.predivide, wl.init_scale, 2.0, 1.0,
-                                        wl.scale_window)
+                                        wl.scale_window, optimizer=1 if optimizer == "sgd" else 0)
         self.scaler = oracle.Scaler(wl.init_scale, 0, 0)
         self.segs = oracle.segments_array(wl.seg_table(), n, wl.weight_decay)
         self.idx = sample_indices(n, wl.segments)
@@ -139,7 +141,12 @@ class FullRun:
 
     def _oracle_apply(self, sub, info):
         wl = self.wl
-        if not info.overflow:
+        if info.overflow:
+            return
+        if self.optimizer == "sgd":
+            oracle.sgd_apply(self.idx.astype(np.uint64), 0, sub, wl.bf16, self.segs, self.s_master, self.s_w,
+                             wl.bf16, self.ohp, wl.lr, info)
+        else:
             oracle.adam_apply(self.idx.astype(np.uint64), 0, sub, wl.bf16, self.segs, self.s_master, self.s_m,
                               self.s_v, self.s_w, wl.bf16, self.ohp, wl.lr, info)
 
@@ -219,11 +226,11 @@ def _free_memory():
     torch.cuda.empty_cache()
 
 
-def _run(wl, steps, exact, check_every=1):
+def _run(wl, steps, exact, check_every=1, optimizer="adamw"):
     """`steps` calls; the state is compared after every `check_every`-th call
     and after the last."""
     t0 = time.time()
-    r = FullRun(wl)
+    r = FullRun(wl, optimizer=optimizer)
     flags, diag = [], {}
     for s in range(1, steps + 1):
         r.gen(s)
@@ -245,6 +252,16 @@ def test_pythia_1p4b_shaped_full_size_exact():
     wl = W.pythia_1p4b()
     r, flags = _run(wl, wl.steps, exact=True)
     assert flags == [0] * wl.steps
+    r.close()
+
+
+def test_pythia_1p4b_shaped_full_size_sgd_exact():
+    """The plain-SGD update over the same 10 calls, bit-exact: master and the
+    16-bit copy follow the oracle's SGD, and m and v stay zero."""
+    wl = W.pythia_1p4b()
+    r, flags = _run(wl, wl.steps, exact=True, optimizer="sgd")
+    assert flags == [0] * wl.steps
+    assert not r.m.t.any().item() and not r.v.t.any().item()
     r.close()
 
 
