@@ -93,14 +93,15 @@ class IpcEventBarrier:
     device collectives (gloo; also several processes on one GPU).
 
     Every rank owns two events that the others open through their IPC
-    handles.  Round r of the barrier on a rank: record its event r mod 2 on
-    the stream; a host barrier over the group (it only tells each rank that
-    the others have *issued* their records, and never waits for the GPU);
-    then the stream waits on every other rank's event r mod 2.  A wait on an
-    event refers to the last record issued before it, hence the host barrier.
-    With two events per rank no rank can record round r + 2 before every rank
-    has issued its waits of round r (that needs the host barrier of round
-    r + 1), so no wait ever takes a later round's record for its own.
+    handles.  Crossing r of the barrier on a rank: record its event r mod 2
+    on the stream; a host barrier over the group (it only tells each rank
+    that the others have *issued* their records, and never waits for the
+    GPU); then the stream waits on every other rank's event r mod 2.  A wait
+    on an event refers to the last record issued before it, hence the host
+    barrier.  With two events per rank no rank can record crossing r + 2
+    before every rank has issued its waits of crossing r (that needs the host
+    barrier of crossing r + 1), so no wait ever takes a later crossing's
+    record for its own.
 
     `event`, `open_event`, `host_barrier` and `exchange` (the all-gather of
     the event handles) are injectable for tests of the protocol without a
@@ -131,14 +132,14 @@ class IpcEventBarrier:
         handles = exchange([e.ipc_handle() for e in self.own])
         self.peers = [[None, None] if r == self.rank else [open_event(h) for h in handles[r]]
                       for r in range(self.world)]
-        self.round = 0
+        self.crossing = 0
 
     def __call__(self, stream=None) -> None:
         if stream is None:
             import torch
             stream = torch.cuda.current_stream()
-        p = self.round & 1
-        self.round += 1
+        p = self.crossing & 1
+        self.crossing += 1
         self.own[p].record(stream)
         self._host_barrier()
         for r in range(self.world):

@@ -1,14 +1,14 @@
 """The ZeRO-2 step's cross-rank ordering, on CPU (gloo, 2 and 3 ranks).
 
 zero.IpcEventBarrier orders the ranks' streams with interprocess CUDA events:
-record this rank's event of the round's parity, a host barrier (only to know
+record this rank's event of the crossing's parity, a host barrier (only to know
 the peers' records are issued), then wait on the peers' events of the same
 parity.  Here the events are stand-ins that keep, in memory shared by the
 ranks, how many records each event has had; a wait notes which record it
-refers to (the last one issued).  Every wait of round r must refer to exactly
-the peers' record of round r -- not an earlier one (the ordering would be
-lost) and not a later one (the wait would stall a round) -- under random
-delays between the calls.  zero2_step's order of operations and its RankLost
+refers to (the last one issued).  Every wait of crossing r must refer to
+exactly the peers' record of crossing r -- not an earlier one (the ordering
+would be lost) and not a later one (the wait would stall a crossing) -- under
+random delays between the calls.  zero2_step's order of operations and its RankLost
 are checked with a stand-in shard.
 """
 import os
@@ -19,7 +19,7 @@ import time
 import pytest
 import torch.multiprocessing as mp
 
-ROUNDS = 12
+CROSSINGS = 12
 
 
 def _free_port():
@@ -68,7 +68,7 @@ def _rank_barrier(rank, world, port, counts, q):
         rng = random.Random(rank * 7919)
         log = []
         stream = _Stream(counts, log)
-        for r in range(ROUNDS):
+        for r in range(CROSSINGS):
             time.sleep(rng.random() * 0.02)
             before = len(log)
             b(stream)
@@ -79,7 +79,7 @@ def _rank_barrier(rank, world, port, counts, q):
 
 
 @pytest.mark.parametrize("world", [2, 3])
-def test_ipc_event_barrier_waits_refer_to_the_same_round(world):
+def test_ipc_event_barrier_waits_refer_to_the_same_crossing(world):
     ctx = mp.get_context("spawn")
     mgr = ctx.Manager()
     counts = mgr.dict()
@@ -88,13 +88,13 @@ def test_ipc_event_barrier_waits_refer_to_the_same_round(world):
     procs = [ctx.Process(target=_rank_barrier, args=(r, world, port, counts, q)) for r in range(world)]
     for p in procs:
         p.start()
-    got = [q.get(timeout=120) for _ in range(world * ROUNDS)]
+    got = [q.get(timeout=120) for _ in range(world * CROSSINGS)]
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
     for rank, r, waits in got:
-        # one wait per other rank and round, on that rank's event of this round's
-        # parity, referring to its (r // 2 + 1)-th record of that event: this round's
+        # one wait per other rank and crossing, on that rank's event of the crossing's
+        # parity, referring to its (r // 2 + 1)-th record of that event: the same crossing's
         assert waits == [((p, r % 2), r // 2 + 1) for p in range(world) if p != rank], (rank, r, waits)
 
 
