@@ -155,3 +155,33 @@ def test_multi_create_rejects_invalid_arguments_before_cuda():
         assert why in L.neox_multi_last_error(None).decode()
     assert L.neox_multi_step(None, 1e-3, None, None) == _abi.NEOX_ERR_INVALID_ARGUMENT
     L.neox_multi_destroy(None)
+
+
+def test_noalloc_rejects_invalid_arguments_before_cuda():
+    """The allocation-free step validates everything before its first CUDA
+    call, so a caller learns of a bad argument without a device: a segment
+    table beyond the static scratch's 1024 entries, a hysteresis count its
+    caller-held scaler state cannot carry, K outside [1, 64], a bad scale.
+    The caller's state is left as it was."""
+    nseg = 1025
+    segs = (_abi.neox_segment * nseg)(*[_abi.neox_segment(4 * i, 4, 0.1) for i in range(nseg)])
+    fake = 0x100000  # never dereferenced: validation fails first
+
+    def desc(n=4 * nseg, with_segs=True):
+        return _abi.neox_shard_desc(n, _abi.NEOX_FP16, _abi.NEOX_FP16,
+                                    ctypes.cast(segs, ctypes.POINTER(_abi.neox_segment)) if with_segs else None,
+                                    nseg if with_segs else 0, 0.1, fake, fake, fake, 1)
+
+    hp = _abi.neox_hparams(0.9, 0.95, 1e-8, 1.0, 1.0, 1024.0, 2.0, 1.0, 1000, 1, 0)
+    hp_hyst = _abi.neox_hparams(0.9, 0.95, 1e-8, 1.0, 1.0, 1024.0, 2.0, 1.0, 1000, 2, 0)
+    cases = [(desc(), hp, 1, 1024.0, "1024"),
+             (desc(with_segs=False), hp_hyst, 1, 1024.0, "hysteresis"),
+             (desc(with_segs=False), hp, 0, 1024.0, "num_grads"),
+             (desc(with_segs=False), hp, 65, 1024.0, "num_grads"),
+             (desc(with_segs=False), hp, 1, 0.0, "scale")]
+    for d, h, k, scale, why in cases:
+        state = _abi.neox_scaler_state(scale, 3, 7)
+        with pytest.raises(_abi.NeoxError) as ei:
+            _abi.neox_shard_step_noalloc(d, h, state, [fake] * k, fake, 1e-3, 0)
+        assert ei.value.status == _abi.NEOX_ERR_INVALID_ARGUMENT and why in str(ei.value), (why, str(ei.value))
+        assert (state.scale, state.good, state.t) == (scale, 3, 7)
