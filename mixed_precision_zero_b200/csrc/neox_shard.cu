@@ -420,7 +420,9 @@ __device__ __forceinline__ void pass2_vectors(const GradPtrs& gp, int K_rt, cons
                         continue;
                     }
                 }
-                const unsigned long long i = L.head + vi * VEC;  // also after the split tiles: they end at element 8 nsplit
+                // contiguous mapping (VEC < 8, or past the whole tiles, which cover
+                // elements head .. head + 8 nsplit - 1)
+                const unsigned long long i = L.head + vi * VEC;
                 float g[VEC], p[VEC], mm[VEC], vv[VEC], keep[VEC];
                 if constexpr (READ_ACC) ld32<VEC>(acc + i, g);
                 else ingest<G, VEC>(gp, K, i, a.inv_pre, inv_us, g);
